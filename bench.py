@@ -1,0 +1,542 @@
+"""Benchmark of the BitLinear forward on B200: one JSON line on rank 0.
+
+Headline workload (the decode metric is quoted on it): the 3B-class decode
+GEMV pair K=3200 -> N=8640 and K=8640 -> N=3200 at M=1 token, bf16
+activations and outputs, latent weights N(0, 0.02^2) packed to 2 bits.
+One step = for each of the two matrices, per-token absmax quantisation
+plus integer accumulation and rescale (the per-token half of the layer;
+packing is load-time and is timed separately under "pack").  Inputs are
+resident in HBM; the packed weights rotate through enough copies that each
+step reads them from HBM, not L2.  ``value`` = algorithmic bytes of the
+step / device time, in GB/s.
+
+Also reported on the same line: "prefill" (7B-class M=2048 GEMM on the
+tensor cores, int8 TOPS vs the int8 peak), "pack" (load-time), "roofline"
+of the dominant kernel, "e2e" through the public API with host buffers,
+"cpu_baseline" (the CPU oracle on the host cores, rank 0 only) and the SM
+clocks seen during the timed region.
+
+--impl reference times the CPU oracle on the same workload (the method's
+reference implementation here), each step a bounded sample of it.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import ctypes  # noqa: E402
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+import torch.distributed as dist  # noqa: E402
+
+METRIC = "BitLinear decode GB/s & %HBM roofline (M=1); prefill int8 TOPS & %peak"
+WORKLOAD = "decode_3b"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+INT8_PER_BF16 = 2.0  # nominal dense ratio (4.5 POPS int8 : 2.25 PFLOP/s bf16)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def decode_bytes(M, K, N, out_bytes=2, in_bytes=2):
+    """Algorithmic bytes of one matrix's per-token step.
+    quant: read x (M*K*in), write x~ (M*K), eta and xsum (8M);
+    forward: read packed W (N*ceil(K/4)), x~ (M*K), eta, xsum (8M), gamma (4),
+    write y (M*N*out)."""
+    quant = M * K * in_bytes + M * K + 8 * M
+    fwd = N * ((K + 3) // 4) + M * K + 8 * M + 4 + M * N * out_bytes
+    return quant, fwd
+
+
+# ----------------------------------------------------------------- distributed plumbing
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1 and not dist.is_initialized():
+        import datetime
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def max_over_ranks(v, world):
+    if world == 1:
+        return v
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([float(v)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        dist.barrier()
+
+
+# ----------------------------------------------------------------- clocks
+
+CLOCK_Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+           "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+           "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+class ClockSampler:
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", "clocks_bench_%d.csv" % os.getpid())
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + CLOCK_Q,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.proc.wait(5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r) if v == "Active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows),
+                "sm_max_mhz": max(r[1] for r in rows), "samples": len(rows), "reasons": reasons}
+
+
+# ----------------------------------------------------------------- our arm
+
+class Capture:
+    """CUDA graph of a list of C-ABI calls, replayed for timing."""
+
+    def __init__(self, calls, stream):
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            with torch.cuda.graph(self.graph, stream=stream):
+                for fn in calls:
+                    fn()
+
+    def replay(self):
+        self.graph.replay()
+
+
+def timed(fn_replays, stream, world):
+    barrier(world)
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    fn_replays()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    return t0.elapsed_time(t1) / 1e3  # seconds
+
+
+def run_ours(args, world, rank, local):
+    from ternary_weight_linear_04_b200 import _lib, build as libbuild, inputs
+    from ternary_weight_linear_04_b200 import bitlinear as bl
+
+    if rank == 0 or world == 1:
+        libbuild.build()
+    barrier(world)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    L = _lib.lib()
+    stream = torch.cuda.Stream(device=dev)
+    sptr = ctypes.c_void_p(stream.cuda_stream)
+    peaks, peak_src = load_peaks()
+    props = torch.cuda.get_device_properties(dev)
+    l2 = getattr(props, "L2_cache_size", 126 * 2 ** 20) or 126 * 2 ** 20
+
+    wl = inputs.WORKLOADS[WORKLOAD]
+    M = args.m
+    mats = []
+    for j, mat in enumerate(wl.matrices):
+        W, x = inputs.make_matrix_inputs(wl, j, m_max=M)
+        Wd = torch.from_numpy(W).to(dev)
+        with torch.cuda.stream(stream):
+            packed, gamma = bl.pack_weights(Wd, stream=stream)
+        xd = torch.from_numpy(x).to(dev).to(torch.bfloat16)
+        mats.append(dict(K=mat.K, N=mat.N, W=Wd, packed=packed, gamma=gamma, x=xd,
+                         xq=torch.empty((M, mat.K), dtype=torch.int8, device=dev),
+                         eta=torch.empty(M, dtype=torch.float32, device=dev),
+                         xsum=torch.empty(M, dtype=torch.int32, device=dev),
+                         y=torch.empty((M, mat.N), dtype=torch.bfloat16, device=dev)))
+    torch.cuda.synchronize()
+    step_w_bytes = sum(m["N"] * ((m["K"] + 3) // 4) for m in mats)
+    copies = max(2, int(np.ceil(3 * l2 / step_w_bytes)))
+    for m in mats:
+        m["copies"] = [(m["packed"], m["gamma"])] + [(m["packed"].clone(), m["gamma"].clone())
+                                                     for _ in range(copies - 1)]
+    torch.cuda.synchronize()
+
+    P = ctypes.c_void_p
+
+    def quant_call(m):
+        args_ = (P(m["x"].data_ptr()), _lib.BL_BF16, M, m["K"], P(m["xq"].data_ptr()),
+                 P(m["eta"].data_ptr()), P(m["xsum"].data_ptr()), sptr)
+        return lambda: _chk(L.bitlinear_quant_act(*args_), "quant")
+
+    def fwd_call(m, c):
+        pk, g = m["copies"][c]
+        args_ = (P(m["xq"].data_ptr()), P(m["eta"].data_ptr()), P(m["xsum"].data_ptr()), M, m["K"],
+                 P(pk.data_ptr()), P(g.data_ptr()), m["N"], P(m["y"].data_ptr()), _lib.BL_BF16,
+                 None, sptr)
+        return lambda: _chk(L.bitlinear_forward(*args_), "forward")
+
+    def step_calls(c):
+        out = []
+        for m in mats:
+            out += [quant_call(m), fwd_call(m, c)]
+        return out
+
+    # Warm-up (also sets kernel attributes outside capture).
+    with torch.cuda.stream(stream):
+        for i in range(max(args.warmup, 3)):
+            for fn in step_calls(i % copies):
+                fn()
+    torch.cuda.synchronize()
+
+    G = copies  # one graph walks every weight copy once
+    full, rem = divmod(args.steps, G)
+    g_full = Capture([fn for c in range(G) for fn in step_calls(c)], stream)
+    g_rem = Capture([fn for c in range(rem) for fn in step_calls(c)], stream) if rem else None
+    # graph warm-up
+    for _ in range(2):
+        g_full.replay()
+    torch.cuda.synchronize()
+
+    def replays():
+        for _ in range(full):
+            g_full.replay()
+        if g_rem:
+            g_rem.replay()
+
+    with ClockSampler(local) as clk:
+        t_step = timed(replays, stream, world)
+        if t_step < 1.0:  # keep the clock sampler's window long enough
+            pass
+    t_step = max_over_ranks(t_step, world)
+    per_step_bytes = 0
+    fwd_bytes = []
+    for m in mats:
+        q, f = decode_bytes(M, m["K"], m["N"])
+        per_step_bytes += q + f
+        fwd_bytes.append(f)
+    value = world * per_step_bytes * args.steps / t_step / 1e9
+    launches = 2 * len(mats) * args.steps
+
+    # Dominant kernel: the accumulate kernel, timed alone the same way.
+    fwd_graph = Capture([fwd_call(m, c) for c in range(G) for m in mats], stream)
+    fwd_graph.replay()
+    torch.cuda.synchronize()
+    reps = max(1, min(full if full else 1, 2000))
+    t_fwd = timed(lambda: [fwd_graph.replay() for _ in range(reps)], stream, world)
+    n_fwd = reps * G * len(mats)
+    avg_fwd = t_fwd / n_fwd
+    achieved = sum(fwd_bytes) / len(mats) / avg_fwd / 1e9
+    hbm_peak = float(peaks["hbm_gbs"])
+    paths = [bl.select_path(M, m["K"], m["N"], m["xq"], m["copies"][0][0], m["y"]) for m in mats]
+    traffic = load_traffic("k_gemv_swar")
+    roofline = {"kernel": "k_gemv_swar (%s path)" % "/".join(sorted(set(paths))),
+                "bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
+                "frac": round(achieved / hbm_peak, 4), "traffic": traffic,
+                "peak_source": peak_src + " hbm_gbs (burst copy)",
+                "avg_launch_us": round(avg_fwd * 1e6, 3),
+                "algorithmic_bytes_per_launch": sum(fwd_bytes) / len(mats)}
+
+    out = {"metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup,
+           "ms_per_step": round(t_step / args.steps * 1e3, 6), "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "int8",
+           "data": "synthetic (seeded N(0,0.02^2) latent weights, N(0,1) bf16 activations)",
+           "config": {"workload": "decode_3b: K=3200->N=8640 and K=8640->N=3200, M=%d, bf16 in/out"
+                                  % M,
+                      "M": M, "parallelism": "replicas" if world > 1 else "single GPU",
+                      "l2": "inputs larger than L2: %d rotating packed-weight copies (%.0f MB > 3x L2)"
+                            % (copies, copies * step_w_bytes / 1e6),
+                      "paths": paths},
+           "roofline": roofline, "gpu_launches": launches,
+           "clocks": clk.summary()}
+
+    if not args.quick:
+        out["e2e"] = run_e2e(args, mats, M, stream, world)
+        out["prefill"] = run_prefill(args, dev, stream, peaks, peak_src, world)
+        out["pack"] = run_pack(mats, stream, world)
+    if (rank == 0) and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = run_cpu_baseline(args.cpu_seconds)
+    return out
+
+
+def _chk(status, what):
+    if status != 0:
+        raise RuntimeError("%s failed with status %d" % (what, status))
+
+
+def load_traffic(kernel):
+    """dram bytes per launch from the committed ncu summary, if present and
+    current (profiles/*.json written alongside the text summaries)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        d = json.load(open(p))
+        return d.get(kernel)
+    except Exception:
+        return None
+
+
+def run_e2e(args, mats, M, stream, world):
+    """Through the public Python API, host buffers in, host buffers out."""
+    from ternary_weight_linear_04_b200 import bitlinear as bl
+    xs_h = [m["x"].cpu().pin_memory() for m in mats]
+    ys_h = [torch.empty_like(m["y"], device="cpu").pin_memory() for m in mats]
+    steps = max(3, min(args.steps, 500))
+    copies = len(mats[0]["copies"])
+
+    def one(i):
+        for j, m in enumerate(mats):
+            pk, g = m["copies"][i % copies]
+            xd = xs_h[j].to(m["x"].device, non_blocking=True)
+            xq, eta, xsum = bl.quant_act(xd, stream=stream)
+            y = bl.forward(xq, eta, xsum, pk, g, m["N"], out_dtype=torch.bfloat16, stream=stream)
+            ys_h[j].copy_(y, non_blocking=True)
+        stream.synchronize()
+
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            one(i)
+        barrier(world)
+        t0 = time.perf_counter()
+        for i in range(steps):
+            one(i)
+        t = time.perf_counter() - t0
+    t = max_over_ranks(t, world)
+    b = sum(sum(decode_bytes(M, m["K"], m["N"])) for m in mats)
+    h2d = sum(M * m["K"] * 2 for m in mats)
+    d2h = sum(M * m["N"] * 2 for m in mats)
+    return {"value": round(world * b * steps / t / 1e9, 2), "unit": "GB/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "ms_per_step": round(t / steps * 1e3, 4), "steps": steps,
+            "note": "public API (bitlinear.quant_act + forward) per step, pinned host x in, "
+                    "host y out, stream synchronised every step"}
+
+
+def run_prefill(args, dev, stream, peaks, peak_src, world):
+    """7B-class prefill: M=2048, K=4096, N=11008 on the tcgen05 path."""
+    from ternary_weight_linear_04_b200 import _lib, inputs
+    from ternary_weight_linear_04_b200 import bitlinear as bl
+    wl = inputs.WORKLOADS["prefill_7b"]
+    W, x = inputs.make_matrix_inputs(wl, 0)
+    M, K, N = x.shape[0], W.shape[1], W.shape[0]
+    with torch.cuda.stream(stream):
+        packed, gamma = bl.pack_weights(torch.from_numpy(W).to(dev), stream=stream)
+        xd = torch.from_numpy(x).to(dev).to(torch.bfloat16)
+        xq, eta, xsum = bl.quant_act(xd, stream=stream)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        for _ in range(3):
+            bl.forward(xq, eta, xsum, packed, gamma, N, stream=stream, out=y)
+    torch.cuda.synchronize()
+    path = bl.select_path(M, K, N, xq, packed, y)
+    reps = 50
+    g = Capture([lambda: bl.forward(xq, eta, xsum, packed, gamma, N, stream=stream, out=y)
+                 for _ in range(10)], stream)
+    g.replay()
+    torch.cuda.synchronize()
+    t = timed(lambda: [g.replay() for _ in range(reps)], stream, world)
+    t = max_over_ranks(t, world)
+    per = t / (reps * 10)
+    ops = 2.0 * M * N * K
+    tops = ops / per / 1e12
+    peak = float(peaks["bf16_tflops"]) * INT8_PER_BF16
+    gq = Capture([lambda: bl.quant_act(xd, stream=stream, out=(xq, eta, xsum)) for _ in range(10)],
+                 stream)
+    gq.replay()
+    torch.cuda.synchronize()
+    tq = timed(lambda: [gq.replay() for _ in range(reps)], stream, world) / (reps * 10)
+    qbytes = M * K * 3 + 8 * M
+    return {"workload": "prefill_7b: M=2048, K=4096, N=11008, bf16 in/out", "path": path,
+            "kernel": "k_gemm_tc", "us_per_forward": round(per * 1e6, 2),
+            "tops": round(tops, 1), "int8_peak_tops": round(peak, 1),
+            "frac": round(tops / peak, 4), "bound": "tensor",
+            "peak_source": "%s bf16_tflops (burst) x %.0f nominal int8:bf16 ratio" % (peak_src, INT8_PER_BF16),
+            "addsub_ops_needed_frac": "nnz(W~)/(N*K) of the dense ops (about 0.69)",
+            "quant_us": round(tq * 1e6, 2), "quant_gbs": round(qbytes / tq / 1e9, 1)}
+
+
+def run_pack(mats, stream, world):
+    from ternary_weight_linear_04_b200 import bitlinear as bl
+    m = mats[0]
+    W = m["W"]
+    N, K = W.shape
+    ws = torch.empty(2048, dtype=torch.uint8, device=W.device)
+    pk = torch.empty_like(m["packed"])
+    g = torch.empty_like(m["gamma"])
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            bl.pack_weights(W, stream=stream, workspace=ws, packed=pk, gamma=g)
+    torch.cuda.synchronize()
+    reps = 20
+    with torch.cuda.stream(stream):
+        t = timed(lambda: [bl.pack_weights(W, stream=stream, workspace=ws, packed=pk, gamma=g)
+                           for _ in range(reps)], stream, world)
+    t = max_over_ranks(t, world) / reps
+    b = 2 * 4 * N * K + N * ((K + 3) // 4)
+    return {"matrix": "%dx%d fp32" % (N, K), "us": round(t * 1e6, 1),
+            "gbs": round(b / t / 1e9, 1),
+            "note": "load-time: exact absmean reduction + ternarise/pack (reads W twice)"}
+
+
+def run_cpu_baseline(seconds):
+    """The CPU oracle (scalar C, OpenMP over output rows) on the same
+    workload, as it stands, for about `seconds` seconds."""
+    from oracle import native as orc
+    from ternary_weight_linear_04_b200 import inputs
+    wl = inputs.WORKLOADS[WORKLOAD]
+    mats = []
+    for j in range(len(wl.matrices)):
+        W, x = inputs.make_matrix_inputs(wl, j, m_max=1)
+        packed, gamma, _ = orc.pack_weights(W)
+        mats.append((W.shape[1], W.shape[0], x, packed, gamma))
+    threads = orc.max_threads()
+    steps = 0
+    t0 = time.perf_counter()
+    while True:
+        for K, N, x, packed, gamma in mats:
+            xq, eta, _ = orc.quant_act(x)
+            orc.forward(xq, eta, packed, gamma, K, N, want_y_int=False)
+        steps += 1
+        if time.perf_counter() - t0 >= seconds:
+            break
+    t = time.perf_counter() - t0
+    b = sum(sum(decode_bytes(1, K, N)) for K, N, *_ in mats)
+    return {"value": round(b * steps / t / 1e9, 4), "unit": "GB/s", "cores": threads,
+            "kind": "oracle",
+            "sample": "%d full decode_3b steps (M=1, both matrices) in %.1f s on %d host threads"
+                      % (steps, t, threads)}
+
+
+# ----------------------------------------------------------------- reference arm
+
+def run_reference(args, world, rank):
+    """The CPU oracle timed on this machine's host cores: each step a bounded
+    sample of the decode workload (a slice of output rows of both
+    matrices), sized so warm-up + steps take about two minutes."""
+    if rank != 0:
+        return None
+    from oracle import native as orc
+    from ternary_weight_linear_04_b200 import inputs
+    wl = inputs.WORKLOADS[WORKLOAD]
+    mats = []
+    for j in range(len(wl.matrices)):
+        W, x = inputs.make_matrix_inputs(wl, j, m_max=args.m)
+        packed, gamma, _ = orc.pack_weights(W)
+        mats.append((W.shape[1], W.shape[0], x, packed, gamma))
+    threads = orc.max_threads()
+
+    def step(frac):
+        tot = 0
+        for K, N, x, packed, gamma in mats:
+            n = max(1, int(N * frac))
+            xq, eta, _ = orc.quant_act(x)
+            orc.forward(xq, eta, packed[:n], gamma, K, n, want_y_int=False)
+            q, f = decode_bytes(x.shape[0], K, n)
+            tot += q + f
+        return tot
+
+    t0 = time.perf_counter()
+    step(1.0)
+    t_full = time.perf_counter() - t0
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    frac = min(1.0, budget / max(t_full, 1e-9))
+    for _ in range(args.warmup):
+        step(frac)
+    b = 0
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        b += step(frac)
+    t = time.perf_counter() - t0
+    value = b / t / 1e9
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(t / args.steps * 1e3, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+            "config": {"workload": "decode_3b: K=3200->N=8640 and K=8640->N=3200, M=%d, bf16 in/out"
+                                   % args.m, "M": args.m},
+            "cpu_baseline": {"kind": "oracle", "cores": threads, "value": round(value, 4),
+                             "unit": "GB/s",
+                             "sample": "each step: %.4f of the output rows of both matrices" % frac},
+            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--m", type=int, default=1, help="tokens per step (decode batch)")
+    ap.add_argument("--quick", action="store_true", help="headline only (no e2e/prefill/pack)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world, rank, local = dist_setup(args.gpus)
+    try:
+        if args.impl == "reference":
+            out = run_reference(args, world, rank)
+        else:
+            out = run_ours(args, world, rank, local)
+        if rank == 0 and out is not None:
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1 and dist.is_initialized():
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,186 @@
+/*
+ * bitlinear.h -- C ABI of the BitNet b1.58 BitLinear forward pass on one
+ * NVIDIA B200 (sm_100a).
+ *
+ * The layer, as the pages define it (cited by title and section):
+ *   [Production]  "BitNet b1.58 & 1-Bit LLMs in Production: Ternary
+ *                 Quantization, MatMul-Free Kernels, and Edge AI Silicon
+ *                 Deployment"
+ *   [Additive]    "1-Bit Large Language Models and BitNet b1.58: How Ternary
+ *                 Weights and Additive Kernels Eliminate Matrix
+ *                 Multiplications"
+ *   [No-Multiply] "BitNet b1.58: Ternary Weight LLMs That Eliminate Matrix
+ *                 Multiplication"
+ *
+ *   gamma   = max(mean |W|, 1e-5)                 whole N x K matrix
+ *   W~      = Clip(Round(W / gamma), -1, +1)      round half to even
+ *   eta_m   = max(max_k |x[m,k]|, 1e-5)           per token m
+ *   x~      = Clip(Round((x * 127) / eta_m), -127, 127)   int8
+ *   y_int   = sum_{W~=+1} x~ - sum_{W~=-1} x~     int32, zeros skipped
+ *   y       = y_int * ((eta_m * gamma) / 127)     fp32, or rounded to bf16
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller (for
+ *     example torch tensors); the library allocates nothing and keeps no
+ *     reference after the call returns.  Scratch space, where one is needed,
+ *     is passed in by the caller.
+ *   - Tensors are dense and row-major: W is N x K (out_features x
+ *     in_features), x and x~ are M x K, y and y_int are M x N.
+ *   - Every call is asynchronous on the CUDA stream `stream` (a cudaStream_t
+ *     passed as void*; NULL = the legacy default stream) and never
+ *     synchronises with the host.  gamma and eta stay on the device.
+ *   - Arguments are checked before anything is launched.  A bad argument
+ *     returns an error status and launches nothing; no call aborts or
+ *     throws.  A CUDA launch error returns BL_ERR_CUDA.  Inputs must be
+ *     finite; NaN or Inf inputs are outside the contract.
+ *   - The results are bit-exact: packed bytes, x~, eta, xsum and y_int
+ *     equal the CPU oracle's exactly, and y is the single fp32 rounding of
+ *     float(y_int) * s_m with s_m = RN32(RN32(eta_m * gamma) / 127).
+ */
+#ifndef BITLINEAR_H
+#define BITLINEAR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    BL_OK = 0,
+    BL_ERR_INVALID_ARG = 1, /* null pointer, negative or zero size, unknown dtype */
+    BL_ERR_UNSUPPORTED = 2, /* sizes beyond the stated limits, or no B200-class GPU */
+    BL_ERR_ALIGNMENT = 3,   /* a pointer breaks the alignment stated for it */
+    BL_ERR_CUDA = 4,        /* a CUDA runtime error at launch time */
+    BL_ERR_TIMEOUT = 5      /* a kernel gave up a bounded wait (see bitlinear_device_error) */
+} bl_status;
+
+typedef enum {
+    BL_F32 = 0,
+    BL_BF16 = 1
+} bl_dtype;
+
+/* Which accumulate kernel bitlinear_forward_path runs. */
+typedef enum {
+    BL_PATH_AUTO = 0,    /* chosen from M, K and alignment (what bitlinear_forward does) */
+    BL_PATH_GEMV = 1,    /* CUDA-core decode kernel, packed weights streamed from HBM */
+    BL_PATH_TCGEN05 = 2, /* tensor-core kernel: tcgen05 kind::i8, accumulators in TMEM */
+    BL_PATH_GENERIC = 3  /* any K, any alignment; plain add/sub/skip per code */
+} bl_path;
+
+/* Human-readable text for a status code (static storage, never NULL). */
+const char* bitlinear_status_str(bl_status status);
+
+/* Bytes of the packed ternary matrix: N * ceil(K/4).  0 if N or K < 1. */
+size_t bitlinear_packed_bytes(int64_t N, int64_t K);
+
+/* Bytes of scratch bitlinear_pack_weights needs (256 exponent buckets of
+ * 64-bit integers, 2048 bytes).  The caller allocates it, 8-byte aligned. */
+size_t bitlinear_pack_workspace_bytes(void);
+
+/*
+ * Load-time half of the layer: absmean ternarisation and 2-bit packing.
+ * [Production] "1. Absmean Weight Quantization" (gamma, Round then Clip) and
+ * WeightQuantizerSTE (clamp at 1e-5); codes from [Production] "Production
+ * Deployment Standards" guideline 1 and [No-Multiply] "Kernel
+ * Implementation: The Lookup Table Approach".
+ *
+ *   W         in   fp32, N x K row-major (leading dimension K).
+ *   N, K      in   out_features >= 1, in_features >= 1, N*K < 2^40.
+ *   packed    out  uint8, N x P with P = ceil(K/4) (bitlinear_packed_bytes):
+ *                  byte n*P + k/4 holds code (W~[n,k] + 1) in bits
+ *                  2*(k%4)..2*(k%4)+1, i.e. 00 = -1, 01 = 0, 10 = +1.
+ *                  Codes past K in the last byte of a row are 01.
+ *   gamma     out  one fp32 on the device: max(RN32(RN64(S) / (N*K)),
+ *                  1e-5) with S the exact sum of |W| (order-independent,
+ *                  so every GPU and the CPU oracle agree to the bit).
+ *   workspace in   bitlinear_pack_workspace_bytes() bytes of device scratch;
+ *                  overwritten; must not be shared by calls that may
+ *                  overlap on the GPU.
+ * Errors: BL_ERR_INVALID_ARG for null pointers or N, K < 1;
+ * BL_ERR_UNSUPPORTED for N*K >= 2^40; BL_ERR_ALIGNMENT if workspace is not
+ * 8-byte or W not 4-byte aligned.
+ */
+bl_status bitlinear_pack_weights(const float* W, int64_t N, int64_t K,
+                                 uint8_t* packed, float* gamma,
+                                 void* workspace, void* stream);
+
+/*
+ * Per-token absmax int8 quantisation of activations.
+ * [Production] "2. Absmax Dynamic Activation Quantization" and
+ * ActivationQuantizerSTE: eta per token (last dimension), clamp at 1e-5,
+ * Round(x * 127 / eta) evaluated as two fp32 roundings in that order.
+ *
+ *   x     in   M x K row-major, fp32 (xdt = BL_F32) or bf16 (BL_BF16).
+ *   M     in   tokens >= 0 (M = 0 is a no-op returning BL_OK).
+ *   K     in   in_features >= 1.
+ *   xq    out  int8, M x K row-major: clip(RNE(RN32(RN32(x*127)/eta_m)), -127, 127).
+ *   eta   out  fp32, M: max(max_k |x[m,k]|, 1e-5).
+ *   xsum  out  int32, M: sum_k xq[m,k] (used by the accumulate kernels);
+ *              may not be NULL.
+ * Errors: BL_ERR_INVALID_ARG for null pointers, M < 0, K < 1 or an unknown
+ * dtype; BL_ERR_ALIGNMENT if x is not aligned to its element size.
+ */
+bl_status bitlinear_quant_act(const void* x, bl_dtype xdt, int64_t M, int64_t K,
+                              int8_t* xq, float* eta, int32_t* xsum, void* stream);
+
+/*
+ * Per-token half of the layer: integer accumulation and rescale.
+ * [Production] "The MatMul-Free Breakthrough" (add where W~ = +1, subtract
+ * where W~ = -1, skip zeros), [Additive] "3. Additive Integer Accumulation",
+ * and [Production] pipeline step 5 / BitLinear158.forward (rescale by
+ * (eta * gamma) / 127).
+ *
+ *   xq, eta, xsum  in   as written by bitlinear_quant_act (M x K, M, M).
+ *   M, K           in   M >= 0 (0 = no-op), K >= 1, 127*K < 2^31.
+ *   packed, gamma  in   as written by bitlinear_pack_weights for N x K.
+ *   N              in   out_features >= 1.
+ *   y              out  M x N row-major, fp32 (ydt = BL_F32) or bf16
+ *                       (BL_BF16, round to nearest even of the fp32 y).
+ *   y_int          out  optional int32 M x N row-major (NULL = not written).
+ * The fast kernels need K % 64 == 0 and 16-byte aligned xq, packed, y and
+ * y_int; other inputs run a generic kernel with the same results.
+ * Errors: BL_ERR_INVALID_ARG for null pointers (other than y_int), N or
+ * K < 1, M < 0 or an unknown dtype; BL_ERR_UNSUPPORTED if 127*K >= 2^31.
+ */
+bl_status bitlinear_forward(const int8_t* xq, const float* eta, const int32_t* xsum,
+                            int64_t M, int64_t K,
+                            const uint8_t* packed, const float* gamma, int64_t N,
+                            void* y, bl_dtype ydt, int32_t* y_int, void* stream);
+
+/*
+ * bitlinear_forward with the accumulate kernel chosen by the caller (for
+ * tests and sweeps).  BL_PATH_GEMV and BL_PATH_TCGEN05 return
+ * BL_ERR_UNSUPPORTED when the inputs do not meet their layout needs
+ * (K % 64 == 0, 16-byte alignment; for BL_PATH_GEMV also M <= 8); the
+ * results of every path are identical.
+ */
+bl_status bitlinear_forward_path(const int8_t* xq, const float* eta, const int32_t* xsum,
+                                 int64_t M, int64_t K,
+                                 const uint8_t* packed, const float* gamma, int64_t N,
+                                 void* y, bl_dtype ydt, int32_t* y_int,
+                                 bl_path path, void* stream);
+
+/* The path bitlinear_forward would pick for these sizes and pointers. */
+bl_path bitlinear_select_path(int64_t M, int64_t K, int64_t N,
+                              const void* xq, const void* packed, const void* y,
+                              const void* y_int);
+
+/*
+ * Reads and clears the library's device-side error word for the current
+ * device (synchronises `stream`).  The tensor-core kernel gives every wait
+ * on a barrier a time limit; a wait that runs out records BL_ERR_TIMEOUT
+ * there and the kernel returns early instead of hanging.  *code receives
+ * BL_OK or BL_ERR_TIMEOUT.  Returns BL_ERR_CUDA if the copy fails.
+ */
+bl_status bitlinear_device_error(int32_t* code, void* stream);
+
+/* Library version as "major.minor.patch" (static storage). */
+const char* bitlinear_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BITLINEAR_H */

@@ -1,0 +1,125 @@
+"""Python binding of the BitLinear C ABI (``include/bitlinear.h``).
+
+Argument marshalling only: torch supplies device memory and the current
+CUDA stream; every step of the layer runs in the library's CUDA kernels.
+Names follow the C entry points: ``pack_weights``, ``quant_act``,
+``forward`` (plus ``BitLinear``, a small holder of one packed matrix).
+"""
+import ctypes
+
+import torch
+
+from . import _lib
+from ._lib import check
+
+PATHS = {"auto": _lib.BL_PATH_AUTO, "gemv": _lib.BL_PATH_GEMV,
+         "tcgen05": _lib.BL_PATH_TCGEN05, "generic": _lib.BL_PATH_GENERIC}
+PATH_NAMES = {v: k for k, v in PATHS.items()}
+_DTYPES = {torch.float32: _lib.BL_F32, torch.bfloat16: _lib.BL_BF16}
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def _require_cuda(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("tensors must be contiguous CUDA tensors")
+
+
+def packed_bytes(N, K):
+    return int(_lib.lib().bitlinear_packed_bytes(N, K))
+
+
+def pack_weights(W, stream=None, workspace=None, packed=None, gamma=None):
+    """fp32 latent weights (N x K, CUDA) -> (packed uint8 N x ceil(K/4), gamma fp32[1])."""
+    _require_cuda(W)
+    if W.dtype != torch.float32 or W.dim() != 2:
+        raise ValueError("W must be a 2-D float32 tensor")
+    N, K = W.shape
+    L = _lib.lib()
+    dev = W.device
+    if packed is None:
+        packed = torch.empty((N, (K + 3) // 4), dtype=torch.uint8, device=dev)
+    if gamma is None:
+        gamma = torch.empty(1, dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = torch.empty(int(L.bitlinear_pack_workspace_bytes()), dtype=torch.uint8, device=dev)
+    check(L.bitlinear_pack_weights(_ptr(W), N, K, _ptr(packed), _ptr(gamma), _ptr(workspace),
+                                   _stream(stream)), "bitlinear_pack_weights")
+    return packed, gamma
+
+
+def quant_act(x, stream=None, out=None):
+    """Activations (M x K, fp32 or bf16, CUDA) -> (xq int8 M x K, eta fp32 M, xsum int32 M)."""
+    _require_cuda(x)
+    if x.dim() != 2 or x.dtype not in _DTYPES:
+        raise ValueError("x must be a 2-D float32 or bfloat16 tensor")
+    M, K = x.shape
+    dev = x.device
+    if out is None:
+        out = (torch.empty((M, K), dtype=torch.int8, device=dev),
+               torch.empty(M, dtype=torch.float32, device=dev),
+               torch.empty(M, dtype=torch.int32, device=dev))
+    xq, eta, xsum = out
+    check(_lib.lib().bitlinear_quant_act(_ptr(x), _DTYPES[x.dtype], M, K, _ptr(xq), _ptr(eta),
+                                         _ptr(xsum), _stream(stream)), "bitlinear_quant_act")
+    return xq, eta, xsum
+
+
+def forward(xq, eta, xsum, packed, gamma, N, out_dtype=torch.bfloat16, want_int=False,
+            path="auto", stream=None, out=None, out_int=None):
+    """Integer accumulation + rescale.  Returns y (M x N), or (y, y_int) if want_int."""
+    _require_cuda(xq, eta, xsum, packed, gamma)
+    M, K = xq.shape
+    if packed.shape != (N, (K + 3) // 4):
+        raise ValueError("packed shape %s does not match N=%d, K=%d" % (tuple(packed.shape), N, K))
+    dev = xq.device
+    y = out if out is not None else torch.empty((M, N), dtype=out_dtype, device=dev)
+    y_int = out_int
+    if want_int and y_int is None:
+        y_int = torch.empty((M, N), dtype=torch.int32, device=dev)
+    check(_lib.lib().bitlinear_forward_path(
+        _ptr(xq), _ptr(eta), _ptr(xsum), M, K, _ptr(packed), _ptr(gamma), N, _ptr(y),
+        _DTYPES[y.dtype], _ptr(y_int), PATHS[path], _stream(stream)), "bitlinear_forward")
+    return (y, y_int) if want_int else y
+
+
+def select_path(M, K, N, xq, packed, y, y_int=None):
+    return PATH_NAMES[int(_lib.lib().bitlinear_select_path(M, K, N, _ptr(xq), _ptr(packed),
+                                                           _ptr(y), _ptr(y_int)))]
+
+
+def device_error(stream=None):
+    code = ctypes.c_int32(0)
+    check(_lib.lib().bitlinear_device_error(ctypes.byref(code), _stream(stream)),
+          "bitlinear_device_error")
+    return int(code.value)
+
+
+class BitLinear:
+    """One packed ternary matrix and its gamma, applied to activations.
+
+    ``BitLinear.from_latent(W)`` packs fp32 latent weights (N x K) once;
+    calling the object quantises x (M x K) per token and runs the integer
+    accumulate + rescale."""
+
+    def __init__(self, packed, gamma, in_features, out_features):
+        self.packed, self.gamma = packed, gamma
+        self.in_features, self.out_features = in_features, out_features
+
+    @classmethod
+    def from_latent(cls, W, stream=None):
+        packed, gamma = pack_weights(W, stream=stream)
+        return cls(packed, gamma, W.shape[1], W.shape[0])
+
+    def __call__(self, x, out_dtype=torch.bfloat16, path="auto", stream=None):
+        xq, eta, xsum = quant_act(x, stream=stream)
+        return forward(xq, eta, xsum, self.packed, self.gamma, self.out_features,
+                       out_dtype=out_dtype, path=path, stream=stream)

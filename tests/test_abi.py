@@ -1,0 +1,99 @@
+"""The C-ABI library loads without a GPU, exports every symbol its header
+declares, and rejects bad arguments before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from ternary_weight_linear_04_b200 import _lib
+from ternary_weight_linear_04_b200 import build as libbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def header_symbols():
+    syms = set()
+    for name in os.listdir(os.path.join(ROOT, "include")):
+        if name.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", name)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            syms |= set(re.findall(r"\b(bitlinear_\w+)\s*\(", text))
+    return syms
+
+
+@pytest.fixture(scope="module")
+def L():
+    libbuild.build()
+    return _lib.lib()
+
+
+def test_library_exports_every_declared_symbol(L):
+    syms = header_symbols()
+    assert len(syms) >= 10
+    for s in syms:
+        assert hasattr(L, s), s
+    assert set(_lib.SIGNATURES) == syms
+
+
+def test_host_only_queries(L):
+    assert L.bitlinear_packed_bytes(3, 5) == 3 * 2
+    assert L.bitlinear_packed_bytes(8640, 3200) == 8640 * 800
+    assert L.bitlinear_packed_bytes(0, 5) == 0
+    assert L.bitlinear_pack_workspace_bytes() == 2048
+    assert L.bitlinear_version().decode().count(".") == 2
+    for st in range(6):
+        assert len(L.bitlinear_status_str(st)) > 0
+
+
+def test_bad_arguments_are_rejected_without_a_launch(L):
+    P = ctypes.c_void_p
+    fake = P(256)  # never dereferenced: validation fails first
+    assert L.bitlinear_pack_weights(None, 4, 4, fake, fake, fake, None) == _lib.BL_ERR_INVALID_ARG
+    assert L.bitlinear_pack_weights(fake, 0, 4, fake, fake, fake, None) == _lib.BL_ERR_INVALID_ARG
+    assert L.bitlinear_pack_weights(fake, 4, -1, fake, fake, fake, None) == _lib.BL_ERR_INVALID_ARG
+    assert L.bitlinear_pack_weights(fake, 1 << 21, 1 << 20, fake, fake, fake, None) == _lib.BL_ERR_UNSUPPORTED
+    assert L.bitlinear_pack_weights(P(258), 4, 4, fake, fake, fake, None) == _lib.BL_ERR_ALIGNMENT
+    assert L.bitlinear_quant_act(None, 0, 1, 4, fake, fake, fake, None) == _lib.BL_ERR_INVALID_ARG
+    assert L.bitlinear_quant_act(fake, 7, 1, 4, fake, fake, fake, None) == _lib.BL_ERR_INVALID_ARG
+    assert L.bitlinear_quant_act(fake, 0, -1, 4, fake, fake, fake, None) == _lib.BL_ERR_INVALID_ARG
+    assert L.bitlinear_quant_act(fake, 0, 1, 0, fake, fake, fake, None) == _lib.BL_ERR_INVALID_ARG
+    assert L.bitlinear_quant_act(P(257), 1, 1, 4, fake, fake, fake, None) == _lib.BL_ERR_ALIGNMENT
+    assert L.bitlinear_quant_act(fake, 0, 0, 4, fake, fake, fake, None) == _lib.BL_OK  # M = 0: no-op
+    fwd = L.bitlinear_forward
+    assert fwd(None, fake, fake, 1, 64, fake, fake, 8, fake, 0, None, None) == _lib.BL_ERR_INVALID_ARG
+    assert fwd(fake, fake, fake, 1, 0, fake, fake, 8, fake, 0, None, None) == _lib.BL_ERR_INVALID_ARG
+    assert fwd(fake, fake, fake, 1, 64, fake, fake, 0, fake, 0, None, None) == _lib.BL_ERR_INVALID_ARG
+    assert fwd(fake, fake, fake, 1, 64, fake, fake, 8, fake, 9, None, None) == _lib.BL_ERR_INVALID_ARG
+    assert fwd(fake, fake, fake, 1, 1 << 25, fake, fake, 8, fake, 0, None, None) == _lib.BL_ERR_UNSUPPORTED
+    assert fwd(fake, P(258), fake, 1, 64, fake, fake, 8, fake, 0, None, None) == _lib.BL_ERR_ALIGNMENT
+    assert fwd(fake, fake, fake, 0, 64, fake, fake, 8, fake, 0, None, None) == _lib.BL_OK
+    assert L.bitlinear_forward_path(fake, fake, fake, 1, 64, fake, fake, 8, fake, 0, None, 9,
+                                    None) == _lib.BL_ERR_INVALID_ARG
+    assert L.bitlinear_device_error(None, None) == _lib.BL_ERR_INVALID_ARG
+
+
+def test_path_selection_is_host_logic(L):
+    P = ctypes.c_void_p
+    a = P(1 << 20)
+    sel = L.bitlinear_select_path
+    assert sel(1, 4096, 4096, a, a, a, None) == _lib.BL_PATH_GEMV
+    assert sel(2048, 4096, 11008, a, a, a, None) == _lib.BL_PATH_TCGEN05
+    assert sel(1, 4095, 4096, a, a, a, None) == _lib.BL_PATH_GENERIC      # ragged K
+    assert sel(1, 4096, 4096, P((1 << 20) + 8), a, a, None) == _lib.BL_PATH_GENERIC  # misaligned
+
+
+def test_product_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(_lib, "_lib", None)
+    with pytest.raises(RuntimeError, match="not built"):
+        _lib.lib()
+
+
+def test_product_does_not_import_the_oracle():
+    pkg = os.path.join(ROOT, "ternary_weight_linear_04_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert "oracle" not in re.sub(r"#.*|//.*", "", text).lower() or f == "inputs.py", f

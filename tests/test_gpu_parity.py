@@ -1,0 +1,254 @@
+"""CUDA path vs. the CPU oracle, element by element, on seeded inputs.
+
+Bar: packed bytes, gamma, x~, eta, xsum and y_int are bit-exact; y (fp32 or
+bf16) is bit-exact as well, which is stricter than the 1-ulp bound the
+method's arithmetic allows, because both sides apply the same single fp32
+rounding to each step (the pinned reading of the rescale).  Every call goes
+through the C ABI (``ternary_weight_linear_04_b200.bitlinear``).
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import native as orc
+from ternary_weight_linear_04_b200 import bitlinear as bl
+from ternary_weight_linear_04_b200 import build as libbuild
+from ternary_weight_linear_04_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+
+DT = {"f32": torch.float32, "bf16": torch.bfloat16}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    libbuild.build()
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    yield
+    assert bl.device_error() == 0
+
+
+def gpu_pack(W):
+    packed, gamma = bl.pack_weights(torch.from_numpy(W).cuda())
+    return packed.cpu().numpy(), np.float32(gamma.cpu().numpy()[0]), packed, gamma
+
+
+def gpu_quant(x, act):
+    xq, eta, xsum = bl.quant_act(torch.from_numpy(x).cuda().to(DT[act]))
+    return xq, eta, xsum
+
+
+def y_bits(y):
+    """Bit patterns of a CPU fp32 / bf16 tensor, for exact comparison."""
+    if y.dtype == torch.bfloat16:
+        return y.view(torch.int16).numpy().view(np.uint16)
+    return y.numpy().view(np.uint32)
+
+
+def oracle_y_bits(y32, out):
+    return orc.f32_to_bf16_bits(y32) if out == "bf16" else y32.view(np.uint32)
+
+
+def check_layer(W, x, act="f32", out="f32", path="auto"):
+    N, K = W.shape
+    ref_packed, ref_gamma, _ = orc.pack_weights(W)
+    packed_h, gamma_h, packed, gamma = gpu_pack(W)
+    assert gamma_h.view(np.uint32) == ref_gamma.view(np.uint32), (gamma_h, ref_gamma)
+    np.testing.assert_array_equal(packed_h, ref_packed)
+    ref_xq, ref_eta, ref_xsum = orc.quant_act(x)
+    xq, eta, xsum = gpu_quant(x, act)
+    np.testing.assert_array_equal(xq.cpu().numpy(), ref_xq)
+    np.testing.assert_array_equal(eta.cpu().numpy().view(np.uint32), ref_eta.view(np.uint32))
+    np.testing.assert_array_equal(xsum.cpu().numpy(), ref_xsum)
+    y, y_int = bl.forward(xq, eta, xsum, packed, gamma, N, out_dtype=DT[out], want_int=True, path=path)
+    ref_yint, ref_y = orc.forward(ref_xq, ref_eta, ref_packed, ref_gamma, K, N)
+    np.testing.assert_array_equal(y_int.cpu().numpy(), ref_yint)
+    np.testing.assert_array_equal(y_bits(y.cpu()), oracle_y_bits(ref_y, out))
+
+
+# ----------------------------------------------------------------- small cases
+
+def test_worked_example_through_the_abi():
+    import json, os
+    g = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "worked_example_2x4.json")))
+    W = np.array(g["W"], np.float32)
+    x = np.array(g["x"], np.float32)
+    packed_h, gamma_h, packed, gamma = gpu_pack(W)
+    assert float(gamma_h) == g["gamma"]
+    np.testing.assert_array_equal(packed_h, g["packed"])
+    xq, eta, xsum = gpu_quant(x, "f32")
+    np.testing.assert_array_equal(xq.cpu().numpy(), g["xq"])
+    for path in ("generic", "auto"):
+        y, y_int = bl.forward(xq, eta, xsum, packed, gamma, 2, out_dtype=torch.bfloat16,
+                              want_int=True, path=path)
+        np.testing.assert_array_equal(y_int.cpu().numpy(), g["y_int"])
+        np.testing.assert_array_equal(y_bits(y.cpu()), g["y_bf16_bits"])
+
+
+@pytest.mark.parametrize("K", [1, 2, 3, 5, 63, 65, 130, 255])
+def test_ragged_k_generic(K):
+    W, x = inputs.make_case(10 + K, 3, K, 37)
+    check_layer(W, x, "f32", "f32", path="auto")
+
+
+@pytest.mark.parametrize("path", ["gemv", "tcgen05", "generic"])
+@pytest.mark.parametrize("M,K,N", [(1, 64, 8), (1, 256, 256), (2, 192, 300), (3, 640, 129),
+                                   (4, 3200, 1000), (8, 1024, 257)])
+@pytest.mark.parametrize("out", ["f32", "bf16"])
+def test_paths_agree_with_oracle(path, M, K, N, out):
+    W, x = inputs.make_case(1000 + M * 7 + K + N, M, K, N, act_dtype="bf16")
+    check_layer(W, x, "bf16", out, path=path)
+
+
+@pytest.mark.parametrize("M", [9, 16, 17, 31, 32, 33, 64, 65, 127, 128, 129, 200, 256, 257, 300])
+def test_tcgen05_token_tiles_and_tails(M):
+    """Every token-tile width (16..256) plus ragged tails in M, N and K
+    (K = 704 = 5.5 stages of 128; N = 389 = 3 tiles + 5 rows)."""
+    W, x = inputs.make_case(2000 + M, M, 704, 389, w_dist="laplace", act_dtype="bf16")
+    check_layer(W, x, "bf16", "bf16", path="tcgen05")
+
+
+def test_long_k_pipeline_wraps():
+    """More K stages than pipeline slots (K = 4096: 32 stages)."""
+    W, x = inputs.make_case(77, 40, 4096, 300, act_dtype="bf16")
+    check_layer(W, x, "bf16", "bf16", path="tcgen05")
+    check_layer(W, x[:3], "bf16", "bf16", path="gemv")
+
+
+def test_all_zero_and_identity_weights():
+    K = 256
+    x = np.random.default_rng(0).normal(0, 1, (5, K)).astype(np.float32)
+    for W in (np.zeros((130, K), np.float32), (K * np.eye(K)).astype(np.float32),
+              (-K * np.eye(K)).astype(np.float32)):
+        for path in ("gemv", "tcgen05", "generic"):
+            check_layer(W, x if path != "gemv" else x[:4], "f32", "f32", path=path)
+
+
+def test_quant_unaligned_and_scalar_paths():
+    """bf16/fp32 rows whose K breaks the 16-byte vector width, and a
+    misaligned base pointer (a column slice), take the scalar loop."""
+    rng = np.random.default_rng(3)
+    for act in ("f32", "bf16"):
+        for K in (7, 13, 100, 1001):
+            x = inputs.draw_activations(rng, 6, K, "student_t_outliers", act)
+            ref = orc.quant_act(x)
+            got = gpu_quant(x, act)
+            for a, b in zip(got, ref):
+                np.testing.assert_array_equal(a.cpu().numpy(), b)
+        big = torch.from_numpy(inputs.draw_activations(rng, 4, 129, "normal", act)).cuda().to(DT[act])
+        xs = big[:, 1:].contiguous()[:, :]  # contiguous copy: aligned
+        off = big.reshape(-1)[1:1 + 4 * 128].reshape(4, 128)  # base offset by one element
+        for t in (xs, off):
+            ref = orc.quant_act(t.float().cpu().numpy())
+            got = bl.quant_act(t)
+            for a, b in zip(got, ref):
+                np.testing.assert_array_equal(a.cpu().numpy(), b)
+
+
+def test_empty_batch_is_a_no_op():
+    W, _ = inputs.make_case(5, 1, 128, 64)
+    _, _, packed, gamma = gpu_pack(W)
+    xq = torch.empty((0, 128), dtype=torch.int8, device="cuda")
+    eta = torch.empty(0, dtype=torch.float32, device="cuda")
+    xsum = torch.empty(0, dtype=torch.int32, device="cuda")
+    y = bl.forward(xq, eta, xsum, packed, gamma, 64)
+    assert y.shape == (0, 64)
+    q = bl.quant_act(torch.empty((0, 128), dtype=torch.bfloat16, device="cuda"))
+    assert q[0].shape == (0, 128)
+
+
+def test_gamma_exact_on_hard_sums():
+    """The exact-sum reduction on inputs where a float reduction in any
+    order would differ: huge dynamic range, ties, subnormals."""
+    rng = np.random.default_rng(8)
+    cases = [
+        (rng.standard_normal((333, 77)) * np.exp2(rng.integers(-126, 100, (333, 77)))).astype(np.float32),
+        np.concatenate([np.full((1, 5), 2.0 ** 53), np.ones((1, 3))], axis=1).astype(np.float32),
+        np.full((64, 64), 2.0 ** -149, np.float32),
+        rng.normal(0, 0.02, (1, 1)).astype(np.float32),
+    ]
+    for W in cases:
+        ref_packed, ref_gamma, _ = orc.pack_weights(W)
+        packed_h, gamma_h, _, _ = gpu_pack(W)
+        assert gamma_h.view(np.uint32) == ref_gamma.view(np.uint32)
+        np.testing.assert_array_equal(packed_h, ref_packed)
+
+
+# ----------------------------------------------------------------- full-size workloads
+
+def sample_positions(M, N, rng, extra_rows=(), extra_cols=()):
+    ms = list(rng.integers(0, M, 3000))
+    ns = list(rng.integers(0, N, 3000))
+    for m in extra_rows:
+        ms += [m] * N
+        ns += list(range(N))
+    for n in extra_cols:
+        ms += list(range(M))
+        ns += [n] * M
+    return np.array(ms, np.int64), np.array(ns, np.int64)
+
+
+def check_full(W, x, batches, out="bf16", rows_full=True):
+    N, K = W.shape
+    rng = np.random.default_rng(N + K)
+    ref_packed, ref_gamma, _ = orc.pack_weights(W)
+    packed_h, gamma_h, packed, gamma = gpu_pack(W)
+    assert gamma_h.view(np.uint32) == ref_gamma.view(np.uint32)
+    np.testing.assert_array_equal(packed_h, ref_packed)
+    del packed_h
+    for M in batches:
+        xm = x[:M]
+        ref_xq, ref_eta, ref_xsum = orc.quant_act(xm)
+        xq, eta, xsum = gpu_quant(xm, "bf16")
+        np.testing.assert_array_equal(xq.cpu().numpy(), ref_xq)
+        np.testing.assert_array_equal(eta.cpu().numpy(), ref_eta)
+        np.testing.assert_array_equal(xsum.cpu().numpy(), ref_xsum)
+        y, y_int = bl.forward(xq, eta, xsum, packed, gamma, N, out_dtype=DT[out], want_int=True)
+        y_int = y_int.cpu().numpy()
+        yb = y_bits(y.cpu())
+        rows = (0, M - 1) if rows_full else ()
+        cols = (0, N - 1, min(127, N - 1), min(128, N - 1))
+        ms, ns = sample_positions(M, N, rng, rows, cols)
+        ref_i, ref_y = orc.forward_at(ref_xq, ref_eta, ref_packed, ref_gamma, K, N, ms, ns)
+        np.testing.assert_array_equal(y_int[ms, ns], ref_i)
+        np.testing.assert_array_equal(yb[ms, ns], oracle_y_bits(ref_y, out))
+        # a property that holds everywhere: y_int row sums against the packed codes
+        # (sum_n y_int[m, n] = sum_k x~[m,k] * sum_n t[n,k]) on one random token
+        m = int(rng.integers(0, M))
+        col_t = np.zeros(K, np.int64)
+        for n0 in range(0, N, 1024):
+            from oracle import reference
+            col_t += reference.unpack2(ref_packed[n0:n0 + 1024], K).astype(np.int64).sum(axis=0)
+        assert int(y_int[m].astype(np.int64).sum()) == int(ref_xq[m].astype(np.int64) @ col_t)
+
+
+def test_full_single_256():
+    w = inputs.WORKLOADS["single_256"]
+    W, x = inputs.make_matrix_inputs(w, 0)
+    check_layer(W, x, "f32", "f32")
+
+
+@pytest.mark.parametrize("idx", [0, 1])
+def test_full_decode_3b(idx):
+    w = inputs.WORKLOADS["decode_3b"]
+    W, x = inputs.make_matrix_inputs(w, idx)
+    check_full(W, x, w.batches)
+
+
+def test_full_prefill_7b():
+    w = inputs.WORKLOADS["prefill_7b"]
+    W, x = inputs.make_matrix_inputs(w, 0)
+    check_full(W, x, w.batches)
+
+
+@pytest.mark.parametrize("idx", range(7))
+def test_full_layer_70b(idx):
+    w = inputs.WORKLOADS["layer_70b"]
+    W, x = inputs.make_matrix_inputs(w, idx)
+    check_full(W, x, w.batches)
+
+
+def test_full_outlier_sweep():
+    w = inputs.WORKLOADS["outlier_sweep"]
+    W, x = inputs.make_matrix_inputs(w, 0)
+    check_full(W, x, w.batches)
