@@ -50,14 +50,11 @@ def load_peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
-def decode_bytes(M, K, N, out_bytes=2, in_bytes=2):
-    """Algorithmic bytes of one matrix's per-token step.
-    quant: read x (M*K*in), write x~ (M*K), eta and xsum (8M);
-    forward: read packed W (N*ceil(K/4)), x~ (M*K), eta, xsum (8M), gamma (4),
-    write y (M*N*out)."""
-    quant = M * K * in_bytes + M * K + 8 * M
-    fwd = N * ((K + 3) // 4) + M * K + 8 * M + 4 + M * N * out_bytes
-    return quant, fwd
+def linear_bytes(M, K, N, out_bytes=2, in_bytes=2):
+    """Algorithmic bytes of the fused per-token layer on one matrix: read the
+    packed weights (N*ceil(K/4)), the activations (M*K*in) and gamma (4),
+    write y (M*N*out).  x~, eta and xsum never leave the chip."""
+    return N * ((K + 3) // 4) + M * K * in_bytes + 4 + M * N * out_bytes
 
 
 # ----------------------------------------------------------------- distributed plumbing
@@ -148,27 +145,34 @@ class ClockSampler:
 # ----------------------------------------------------------------- our arm
 
 class Capture:
-    """CUDA graph of a list of C-ABI calls, replayed for timing."""
+    """CUDA graph of a list of C-ABI calls, replayed for timing.  replay()
+    launches on the current stream: callers time it inside timed(), which
+    makes the timed stream current."""
 
     def __init__(self, calls, stream):
         self.graph = torch.cuda.CUDAGraph()
+        self.stream = stream
         with torch.cuda.stream(stream):
             with torch.cuda.graph(self.graph, stream=stream):
                 for fn in calls:
                     fn()
 
     def replay(self):
+        assert torch.cuda.current_stream() == self.stream, "replay on the timed stream"
         self.graph.replay()
 
 
 def timed(fn_replays, stream, world):
+    """Device time of fn_replays(): events recorded on `stream`, and the work
+    (graph replays, library calls) issued on that same stream."""
     barrier(world)
     torch.cuda.synchronize()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    fn_replays()
-    t1.record(stream)
+    with torch.cuda.stream(stream):
+        t0.record(stream)
+        fn_replays()
+        t1.record(stream)
     torch.cuda.synchronize()
     barrier(world)
     return t0.elapsed_time(t1) / 1e3  # seconds
@@ -214,23 +218,18 @@ def run_ours(args, world, rank, local):
 
     P = ctypes.c_void_p
 
-    def quant_call(m):
-        args_ = (P(m["x"].data_ptr()), _lib.BL_BF16, M, m["K"], P(m["xq"].data_ptr()),
-                 P(m["eta"].data_ptr()), P(m["xsum"].data_ptr()), sptr)
-        return lambda: _chk(L.bitlinear_quant_act(*args_), "quant")
-
-    def fwd_call(m, c):
+    def linear_call(m, c):
+        """One call of the whole per-token layer (bitlinear_linear): quantise,
+        accumulate, rescale; weights packed at load time are static."""
         pk, g = m["copies"][c]
-        args_ = (P(m["xq"].data_ptr()), P(m["eta"].data_ptr()), P(m["xsum"].data_ptr()), M, m["K"],
-                 P(pk.data_ptr()), P(g.data_ptr()), m["N"], P(m["y"].data_ptr()), _lib.BL_BF16,
-                 None, sptr)
-        return lambda: _chk(L.bitlinear_forward(*args_), "forward")
+        args_ = (P(m["x"].data_ptr()), _lib.BL_BF16, M, m["K"], P(pk.data_ptr()), P(g.data_ptr()),
+                 m["N"], P(m["y"].data_ptr()), _lib.BL_BF16, P(m["xq"].data_ptr()),
+                 P(m["eta"].data_ptr()), P(m["xsum"].data_ptr()), None,
+                 _lib.BL_FLAG_WEIGHTS_STATIC, sptr)
+        return lambda: _chk(L.bitlinear_linear(*args_), "linear")
 
     def step_calls(c):
-        out = []
-        for m in mats:
-            out += [quant_call(m), fwd_call(m, c)]
-        return out
+        return [linear_call(m, c) for m in mats]
 
     # Warm-up (also sets kernel attributes outside capture).
     with torch.cuda.stream(stream):
@@ -244,8 +243,9 @@ def run_ours(args, world, rank, local):
     g_full = Capture([fn for c in range(G) for fn in step_calls(c)], stream)
     g_rem = Capture([fn for c in range(rem) for fn in step_calls(c)], stream) if rem else None
     # graph warm-up
-    for _ in range(2):
-        g_full.replay()
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            g_full.replay()
     torch.cuda.synchronize()
 
     def replays():
@@ -259,33 +259,23 @@ def run_ours(args, world, rank, local):
         if t_step < 1.0:  # keep the clock sampler's window long enough
             pass
     t_step = max_over_ranks(t_step, world)
-    per_step_bytes = 0
-    fwd_bytes = []
-    for m in mats:
-        q, f = decode_bytes(M, m["K"], m["N"])
-        per_step_bytes += q + f
-        fwd_bytes.append(f)
+    per_step_bytes = sum(linear_bytes(M, m["K"], m["N"]) for m in mats)
     value = world * per_step_bytes * args.steps / t_step / 1e9
-    launches = 2 * len(mats) * args.steps
+    launches = len(mats) * args.steps  # one fused decode kernel per matrix
 
-    # Dominant kernel: the accumulate kernel, timed alone the same way.
-    fwd_graph = Capture([fwd_call(m, c) for c in range(G) for m in mats], stream)
-    fwd_graph.replay()
-    torch.cuda.synchronize()
-    reps = max(1, min(full if full else 1, 2000))
-    t_fwd = timed(lambda: [fwd_graph.replay() for _ in range(reps)], stream, world)
-    n_fwd = reps * G * len(mats)
-    avg_fwd = t_fwd / n_fwd
-    achieved = sum(fwd_bytes) / len(mats) / avg_fwd / 1e9
+    # The step is nothing but the dominant kernel (k_decode, one launch per
+    # matrix), so its per-launch time is the timed region / launches.
+    avg_launch = t_step / launches
+    bytes_per_launch = per_step_bytes / len(mats)
+    achieved = bytes_per_launch / avg_launch / 1e9
     hbm_peak = float(peaks["hbm_gbs"])
     paths = [bl.select_path(M, m["K"], m["N"], m["xq"], m["copies"][0][0], m["y"]) for m in mats]
-    traffic = load_traffic("k_gemv_swar")
-    roofline = {"kernel": "k_gemv_swar (%s path)" % "/".join(sorted(set(paths))),
+    roofline = {"kernel": "k_decode (fused quantise + accumulate + rescale)",
                 "bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
-                "frac": round(achieved / hbm_peak, 4), "traffic": traffic,
+                "frac": round(achieved / hbm_peak, 4), "traffic": load_traffic("k_decode"),
                 "peak_source": peak_src + " hbm_gbs (burst copy)",
-                "avg_launch_us": round(avg_fwd * 1e6, 3),
-                "algorithmic_bytes_per_launch": sum(fwd_bytes) / len(mats)}
+                "avg_launch_us": round(avg_launch * 1e6, 3),
+                "algorithmic_bytes_per_launch": bytes_per_launch}
 
     out = {"metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
            "steps": args.steps, "warmup": args.warmup,
@@ -340,8 +330,8 @@ def run_e2e(args, mats, M, stream, world):
         for j, m in enumerate(mats):
             pk, g = m["copies"][i % copies]
             xd = xs_h[j].to(m["x"].device, non_blocking=True)
-            xq, eta, xsum = bl.quant_act(xd, stream=stream)
-            y = bl.forward(xq, eta, xsum, pk, g, m["N"], out_dtype=torch.bfloat16, stream=stream)
+            y = bl.linear(xd, pk, g, m["N"], out_dtype=torch.bfloat16, weights_static=True,
+                          stream=stream)
             ys_h[j].copy_(y, non_blocking=True)
         stream.synchronize()
 
@@ -354,13 +344,13 @@ def run_e2e(args, mats, M, stream, world):
             one(i)
         t = time.perf_counter() - t0
     t = max_over_ranks(t, world)
-    b = sum(sum(decode_bytes(M, m["K"], m["N"])) for m in mats)
+    b = sum(linear_bytes(M, m["K"], m["N"]) for m in mats)
     h2d = sum(M * m["K"] * 2 for m in mats)
     d2h = sum(M * m["N"] * 2 for m in mats)
     return {"value": round(world * b * steps / t / 1e9, 2), "unit": "GB/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "ms_per_step": round(t / steps * 1e3, 4), "steps": steps,
-            "note": "public API (bitlinear.quant_act + forward) per step, pinned host x in, "
+            "note": "public API (bitlinear.linear) per matrix, pinned host x in, "
                     "host y out, stream synchronised every step"}
 
 
@@ -383,7 +373,8 @@ def run_prefill(args, dev, stream, peaks, peak_src, world):
     reps = 50
     g = Capture([lambda: bl.forward(xq, eta, xsum, packed, gamma, N, stream=stream, out=y)
                  for _ in range(10)], stream)
-    g.replay()
+    with torch.cuda.stream(stream):
+        g.replay()
     torch.cuda.synchronize()
     t = timed(lambda: [g.replay() for _ in range(reps)], stream, world)
     t = max_over_ranks(t, world)
@@ -393,7 +384,8 @@ def run_prefill(args, dev, stream, peaks, peak_src, world):
     peak = float(peaks["bf16_tflops"]) * INT8_PER_BF16
     gq = Capture([lambda: bl.quant_act(xd, stream=stream, out=(xq, eta, xsum)) for _ in range(10)],
                  stream)
-    gq.replay()
+    with torch.cuda.stream(stream):
+        gq.replay()
     torch.cuda.synchronize()
     tq = timed(lambda: [gq.replay() for _ in range(reps)], stream, world) / (reps * 10)
     qbytes = M * K * 3 + 8 * M
@@ -451,7 +443,7 @@ def run_cpu_baseline(seconds):
         if time.perf_counter() - t0 >= seconds:
             break
     t = time.perf_counter() - t0
-    b = sum(sum(decode_bytes(1, K, N)) for K, N, *_ in mats)
+    b = sum(linear_bytes(1, K, N) for K, N, *_ in mats)
     return {"value": round(b * steps / t / 1e9, 4), "unit": "GB/s", "cores": threads,
             "kind": "oracle",
             "sample": "%d full decode_3b steps (M=1, both matrices) in %.1f s on %d host threads"
@@ -482,8 +474,7 @@ def run_reference(args, world, rank):
             n = max(1, int(N * frac))
             xq, eta, _ = orc.quant_act(x)
             orc.forward(xq, eta, packed[:n], gamma, K, n, want_y_int=False)
-            q, f = decode_bytes(x.shape[0], K, n)
-            tot += q + f
+            tot += linear_bytes(x.shape[0], K, n)
         return tot
 
     t0 = time.perf_counter()

@@ -113,7 +113,8 @@ bl_status bitlinear_pack_weights(const float* W, int64_t N, int64_t K,
  * Round(x * 127 / eta) evaluated as two fp32 roundings in that order.
  *
  *   x     in   M x K row-major, fp32 (xdt = BL_F32) or bf16 (BL_BF16).
- *   M     in   tokens >= 0 (M = 0 is a no-op returning BL_OK).
+ *   M     in   tokens >= 0 (M = 0 is a no-op returning BL_OK; the M-sized
+ *              buffers may then be NULL).
  *   K     in   in_features >= 1.
  *   xq    out  int8, M x K row-major: clip(RNE(RN32(RN32(x*127)/eta_m)), -127, 127).
  *   eta   out  fp32, M: max(max_k |x[m,k]|, 1e-5).
@@ -133,7 +134,8 @@ bl_status bitlinear_quant_act(const void* x, bl_dtype xdt, int64_t M, int64_t K,
  * (eta * gamma) / 127).
  *
  *   xq, eta, xsum  in   as written by bitlinear_quant_act (M x K, M, M).
- *   M, K           in   M >= 0 (0 = no-op), K >= 1, 127*K < 2^31.
+ *   M, K           in   M >= 0 (0 = no-op; xq, eta, xsum, y may then be
+ *                       NULL), K >= 1, 127*K < 2^31.
  *   packed, gamma  in   as written by bitlinear_pack_weights for N x K.
  *   N              in   out_features >= 1.
  *   y              out  M x N row-major, fp32 (ydt = BL_F32) or bf16
@@ -150,17 +152,52 @@ bl_status bitlinear_forward(const int8_t* xq, const float* eta, const int32_t* x
                             void* y, bl_dtype ydt, int32_t* y_int, void* stream);
 
 /*
- * bitlinear_forward with the accumulate kernel chosen by the caller (for
- * tests and sweeps).  BL_PATH_GEMV and BL_PATH_TCGEN05 return
- * BL_ERR_UNSUPPORTED when the inputs do not meet their layout needs
- * (K % 64 == 0, 16-byte alignment; for BL_PATH_GEMV also M <= 8); the
- * results of every path are identical.
+ * Flag for bitlinear_forward_path and bitlinear_linear: the caller promises
+ * that `packed` and `gamma` are not written by any work still pending on
+ * `stream` (true for weights packed earlier and synchronised, the normal
+ * inference case).  The decode kernel may then start streaming the packed
+ * weights before the preceding kernel on the stream has finished
+ * (programmatic dependent launch); activations are always read only after
+ * it has finished.
+ */
+#define BL_FLAG_WEIGHTS_STATIC 1u
+
+/*
+ * bitlinear_forward with the accumulate kernel and flags chosen by the
+ * caller.  BL_PATH_GEMV and BL_PATH_TCGEN05 return BL_ERR_UNSUPPORTED when
+ * the inputs do not meet their layout needs (K % 64 == 0, 16-byte
+ * alignment; for BL_PATH_GEMV also M <= 8, K <= 65536 and M*K <= 147456); the results of
+ * every path are identical.  flags: 0 or BL_FLAG_WEIGHTS_STATIC.
  */
 bl_status bitlinear_forward_path(const int8_t* xq, const float* eta, const int32_t* xsum,
                                  int64_t M, int64_t K,
                                  const uint8_t* packed, const float* gamma, int64_t N,
                                  void* y, bl_dtype ydt, int32_t* y_int,
-                                 bl_path path, void* stream);
+                                 bl_path path, unsigned flags, void* stream);
+
+/*
+ * The whole per-token layer in one call: quantise x per token
+ * ([Production] "2. Absmax Dynamic Activation Quantization"), accumulate
+ * with add / subtract / skip ([Production] "The MatMul-Free Breakthrough")
+ * and rescale ([Production] pipeline step 5).  Same results, bit for bit, as
+ * bitlinear_quant_act followed by bitlinear_forward.
+ *
+ *   x, xdt, M, K      in   activations as for bitlinear_quant_act.
+ *   packed, gamma, N  in   as for bitlinear_forward.
+ *   y, ydt, y_int     out  as for bitlinear_forward (y_int optional).
+ *   xq, eta, xsum     out  the quantised activations (M x K int8, M fp32,
+ *                          M int32).  For decode batches (M <= 4, K % 64 ==
+ *                          0, 16-byte aligned x, packed, y) one fused kernel
+ *                          runs and these are optional (NULL = not written).
+ *                          Otherwise two kernels run and they are required
+ *                          scratch (BL_ERR_INVALID_ARG if NULL).
+ *   flags             in   0 or BL_FLAG_WEIGHTS_STATIC.
+ */
+bl_status bitlinear_linear(const void* x, bl_dtype xdt, int64_t M, int64_t K,
+                           const uint8_t* packed, const float* gamma, int64_t N,
+                           void* y, bl_dtype ydt,
+                           int8_t* xq, float* eta, int32_t* xsum,
+                           int32_t* y_int, unsigned flags, void* stream);
 
 /* The path bitlinear_forward would pick for these sizes and pointers. */
 bl_path bitlinear_select_path(int64_t M, int64_t K, int64_t N,

@@ -9,7 +9,7 @@ __version__ = "0.1.0"
 
 
 def __getattr__(name):
-    if name in ("pack_weights", "quant_act", "forward", "BitLinear", "packed_bytes",
+    if name in ("pack_weights", "quant_act", "forward", "linear", "BitLinear", "packed_bytes",
                 "select_path", "device_error"):
         from . import bitlinear
         return getattr(bitlinear, name)

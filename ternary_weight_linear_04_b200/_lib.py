@@ -13,6 +13,7 @@ LIB_PATH = os.path.join(HERE, "libbitlinear.so")
 BL_OK, BL_ERR_INVALID_ARG, BL_ERR_UNSUPPORTED, BL_ERR_ALIGNMENT, BL_ERR_CUDA, BL_ERR_TIMEOUT = range(6)
 BL_F32, BL_BF16 = 0, 1
 BL_PATH_AUTO, BL_PATH_GEMV, BL_PATH_TCGEN05, BL_PATH_GENERIC = range(4)
+BL_FLAG_WEIGHTS_STATIC = 1
 
 # name -> (restype, argtypes); every symbol include/bitlinear.h declares.
 _P = ctypes.c_void_p
@@ -26,7 +27,10 @@ SIGNATURES = {
     "bitlinear_pack_weights": (_I, [_P, _I64, _I64, _P, _P, _P, _P]),
     "bitlinear_quant_act": (_I, [_P, _I, _I64, _I64, _P, _P, _P, _P]),
     "bitlinear_forward": (_I, [_P, _P, _P, _I64, _I64, _P, _P, _I64, _P, _I, _P, _P]),
-    "bitlinear_forward_path": (_I, [_P, _P, _P, _I64, _I64, _P, _P, _I64, _P, _I, _P, _I, _P]),
+    "bitlinear_forward_path": (_I, [_P, _P, _P, _I64, _I64, _P, _P, _I64, _P, _I, _P, _I,
+                                    ctypes.c_uint, _P]),
+    "bitlinear_linear": (_I, [_P, _I, _I64, _I64, _P, _P, _I64, _P, _I, _P, _P, _P, _P,
+                              ctypes.c_uint, _P]),
     "bitlinear_select_path": (_I, [_I64, _I64, _I64, _P, _P, _P, _P]),
     "bitlinear_device_error": (_I, [_P, _P]),
 }

@@ -74,8 +74,10 @@ def quant_act(x, stream=None, out=None):
 
 
 def forward(xq, eta, xsum, packed, gamma, N, out_dtype=torch.bfloat16, want_int=False,
-            path="auto", stream=None, out=None, out_int=None):
-    """Integer accumulation + rescale.  Returns y (M x N), or (y, y_int) if want_int."""
+            path="auto", stream=None, out=None, out_int=None, weights_static=False):
+    """Integer accumulation + rescale.  Returns y (M x N), or (y, y_int) if want_int.
+    weights_static: packed/gamma are not written by pending work on the stream
+    (lets the decode kernel start streaming them early)."""
     _require_cuda(xq, eta, xsum, packed, gamma)
     M, K = xq.shape
     if packed.shape != (N, (K + 3) // 4):
@@ -87,8 +89,43 @@ def forward(xq, eta, xsum, packed, gamma, N, out_dtype=torch.bfloat16, want_int=
         y_int = torch.empty((M, N), dtype=torch.int32, device=dev)
     check(_lib.lib().bitlinear_forward_path(
         _ptr(xq), _ptr(eta), _ptr(xsum), M, K, _ptr(packed), _ptr(gamma), N, _ptr(y),
-        _DTYPES[y.dtype], _ptr(y_int), PATHS[path], _stream(stream)), "bitlinear_forward")
+        _DTYPES[y.dtype], _ptr(y_int), PATHS[path],
+        _lib.BL_FLAG_WEIGHTS_STATIC if weights_static else 0, _stream(stream)), "bitlinear_forward")
     return (y, y_int) if want_int else y
+
+
+def linear(x, packed, gamma, N, out_dtype=torch.bfloat16, want_quant=False, want_int=False,
+           weights_static=False, stream=None, out=None, scratch=None):
+    """The whole per-token layer (quantise + accumulate + rescale) in one call.
+    Returns y, plus (xq, eta, xsum) if want_quant and y_int if want_int."""
+    _require_cuda(x, packed, gamma)
+    if x.dim() != 2 or x.dtype not in _DTYPES:
+        raise ValueError("x must be a 2-D float32 or bfloat16 tensor")
+    M, K = x.shape
+    if packed.shape != (N, (K + 3) // 4):
+        raise ValueError("packed shape %s does not match N=%d, K=%d" % (tuple(packed.shape), N, K))
+    dev = x.device
+    y = out if out is not None else torch.empty((M, N), dtype=out_dtype, device=dev)
+    decode = M <= 4 and K % 64 == 0
+    if scratch is not None:
+        xq, eta, xsum = scratch
+    elif want_quant or not decode:
+        xq = torch.empty((M, K), dtype=torch.int8, device=dev)
+        eta = torch.empty(M, dtype=torch.float32, device=dev)
+        xsum = torch.empty(M, dtype=torch.int32, device=dev)
+    else:
+        xq = eta = xsum = None
+    y_int = torch.empty((M, N), dtype=torch.int32, device=dev) if want_int else None
+    check(_lib.lib().bitlinear_linear(
+        _ptr(x), _DTYPES[x.dtype], M, K, _ptr(packed), _ptr(gamma), N, _ptr(y), _DTYPES[y.dtype],
+        _ptr(xq), _ptr(eta), _ptr(xsum), _ptr(y_int),
+        _lib.BL_FLAG_WEIGHTS_STATIC if weights_static else 0, _stream(stream)), "bitlinear_linear")
+    out_ = (y,)
+    if want_quant:
+        out_ += ((xq, eta, xsum),)
+    if want_int:
+        out_ += (y_int,)
+    return out_[0] if len(out_) == 1 else out_
 
 
 def select_path(M, K, N, xq, packed, y, y_int=None):
@@ -119,7 +156,6 @@ class BitLinear:
         packed, gamma = pack_weights(W, stream=stream)
         return cls(packed, gamma, W.shape[1], W.shape[0])
 
-    def __call__(self, x, out_dtype=torch.bfloat16, path="auto", stream=None):
-        xq, eta, xsum = quant_act(x, stream=stream)
-        return forward(xq, eta, xsum, self.packed, self.gamma, self.out_features,
-                       out_dtype=out_dtype, path=path, stream=stream)
+    def __call__(self, x, out_dtype=torch.bfloat16, stream=None):
+        return linear(x, self.packed, self.gamma, self.out_features, out_dtype=out_dtype,
+                      weights_static=True, stream=stream)

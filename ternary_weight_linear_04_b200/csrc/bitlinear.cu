@@ -10,9 +10,11 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "bitlinear.h"
 #include "common.cuh"
+#include "decode.cuh"
 #include "gemm_tc.cuh"
 #include "gemv.cuh"
 #include "pack.cuh"
@@ -21,9 +23,10 @@
 namespace {
 
 constexpr int kMaxDevices = 64;
-constexpr int kGemvMaxM = 8;          // largest token count the CUDA-core kernel takes
+constexpr int kGemvMaxM = 8;          // largest token count the CUDA-core decode kernel takes
 constexpr int kGemvAutoMaxM = 4;      // auto dispatch: above this, tensor cores
-constexpr int64_t kGemvMaxSmem = 200 * 1024;
+constexpr int64_t kGemvMaxXBytes = 144 * 1024;  // M*K activation bytes the decode kernel stages
+constexpr int64_t kGemvMaxK = 4 * bl::kDecStageBytes;      // a stage holds at least one packed row
 
 inline bool aligned(const void* p, uintptr_t a) {
   return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0;
@@ -34,6 +37,30 @@ inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s
 bl_status launch_status() {
   const cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? BL_OK : BL_ERR_CUDA;
+}
+
+// Launch with programmatic dependent launch allowed: the kernel may start
+// while the previous kernel on the stream finishes; every such kernel calls
+// griddepcontrol.wait before it reads anything an earlier kernel wrote.
+template <typename... KArgs, typename... Args>
+bl_status launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                     Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    return BL_ERR_CUDA;
+  }
+  return launch_status();
 }
 
 // Once per device: is it an sm_100 part, and how many SMs does it have.
@@ -113,43 +140,29 @@ bool make_tmap_u8(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t col
 
 // ------------------------------------------------------------ launchers
 
-template <int MT, int R, typename OutT>
-bl_status launch_gemv_swar(const int8_t* xq, const float* eta, const int32_t* xsum, int M, int K,
-                           const uint8_t* packed, const float* gamma, int N, void* y,
-                           int32_t* y_int, int sms, cudaStream_t st) {
+// Decode kernel (M <= 8 tokens): one CTA per SM-slot, each owning a
+// contiguous block of rows.  FUSED = quantise x inside the kernel.
+template <int MT, bool FUSED, typename XT, typename OutT>
+bl_status launch_decode_mt(const bl::DecodeArgs& a, int sms, cudaStream_t st) {
   static int smem_done[kMaxDevices] = {0};
-  const size_t smem = static_cast<size_t>(MT) * K;
-  auto kern = bl::k_gemv_swar<MT, R, OutT>;
+  const size_t smem = bl::DecSmem<MT>::bytes(a.K);
+  auto kern = bl::k_decode<MT, FUSED, XT, OutT>;
   if (!ensure_smem(kern, smem, smem_done)) return BL_ERR_CUDA;
-  const int warps_per_cta = 8;
-  int64_t ctas = (static_cast<int64_t>(N) + warps_per_cta * R - 1) / (warps_per_cta * R);
-  const int64_t cap = static_cast<int64_t>(sms) * 16;
-  if (ctas > cap) ctas = cap;
-  kern<<<static_cast<int>(ctas), 256, smem, st>>>(xq, eta, xsum, M, K, packed, gamma, N, y, y_int);
-  return launch_status();
+  int64_t grid = static_cast<int64_t>(sms) * bl::DecOcc<MT>::kCtasPerSm;
+  const int64_t max_ctas = (static_cast<int64_t>(a.N) + 3) / 4;
+  if (grid > max_ctas) grid = max_ctas;
+  bl::DecodeArgs args = a;
+  args.rows_per_cta = static_cast<int>((a.N + grid - 1) / grid);
+  grid = (a.N + args.rows_per_cta - 1) / args.rows_per_cta;
+  return launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(bl::kDecThreads), smem, st, args);
 }
 
-template <int MT, typename OutT>
-bl_status gemv_pick_r(const int8_t* xq, const float* eta, const int32_t* xsum, int M, int K,
-                      const uint8_t* packed, const float* gamma, int N, void* y, int32_t* y_int,
-                      int sms, cudaStream_t st) {
-  // Enough warp tasks to fill every SM twice over with 8-warp CTAs.
-  const int64_t want = static_cast<int64_t>(sms) * 16;
-  if (N / 4 >= want)
-    return launch_gemv_swar<MT, 4, OutT>(xq, eta, xsum, M, K, packed, gamma, N, y, y_int, sms, st);
-  if (N / 2 >= want)
-    return launch_gemv_swar<MT, 2, OutT>(xq, eta, xsum, M, K, packed, gamma, N, y, y_int, sms, st);
-  return launch_gemv_swar<MT, 1, OutT>(xq, eta, xsum, M, K, packed, gamma, N, y, y_int, sms, st);
-}
-
-template <typename OutT>
-bl_status launch_gemv(const int8_t* xq, const float* eta, const int32_t* xsum, int M, int K,
-                      const uint8_t* packed, const float* gamma, int N, void* y, int32_t* y_int,
-                      int sms, cudaStream_t st) {
-  if (M <= 1) return gemv_pick_r<1, OutT>(xq, eta, xsum, M, K, packed, gamma, N, y, y_int, sms, st);
-  if (M <= 2) return gemv_pick_r<2, OutT>(xq, eta, xsum, M, K, packed, gamma, N, y, y_int, sms, st);
-  if (M <= 4) return gemv_pick_r<4, OutT>(xq, eta, xsum, M, K, packed, gamma, N, y, y_int, sms, st);
-  return gemv_pick_r<8, OutT>(xq, eta, xsum, M, K, packed, gamma, N, y, y_int, sms, st);
+template <bool FUSED, typename XT, typename OutT>
+bl_status launch_decode(const bl::DecodeArgs& a, int sms, cudaStream_t st) {
+  if (a.M <= 1) return launch_decode_mt<1, FUSED, XT, OutT>(a, sms, st);
+  if (a.M <= 2) return launch_decode_mt<2, FUSED, XT, OutT>(a, sms, st);
+  if (a.M <= 4) return launch_decode_mt<4, FUSED, XT, OutT>(a, sms, st);
+  return launch_decode_mt<8, FUSED, XT, OutT>(a, sms, st);
 }
 
 template <typename OutT>
@@ -163,11 +176,10 @@ bl_status launch_generic(const int8_t* xq, const float* eta, int64_t M, int64_t 
     if (ctas > static_cast<int64_t>(sms) * 16) ctas = static_cast<int64_t>(sms) * 16;
     dim3 grid(static_cast<unsigned>(ctas), static_cast<unsigned>(mb));
     const int64_t m_off = mb0 * 8;
-    bl::k_gemv_generic<OutT><<<grid, 256, 0, st>>>(xq + m_off * K, eta + m_off, M - m_off, K,
-                                                    packed, gamma, N,
-                                                    static_cast<char*>(y) + m_off * N * sizeof(OutT),
-                                                    y_int ? y_int + m_off * N : nullptr);
-    const bl_status s = launch_status();
+    const bl_status s = launch_pdl(
+        bl::k_gemv_generic<OutT>, grid, dim3(256), 0, st, xq + m_off * K, eta + m_off, M - m_off,
+        K, packed, gamma, N, static_cast<void*>(static_cast<char*>(y) + m_off * N * sizeof(OutT)),
+        y_int ? y_int + m_off * N : static_cast<int32_t*>(nullptr));
     if (s != BL_OK) return s;
   }
   return BL_OK;
@@ -188,8 +200,7 @@ bl_status launch_tc_bm(const int8_t* xq, const float* eta, int M, int K, const u
     return BL_ERR_CUDA;
   dim3 grid((N + bl::kTcBN - 1) / bl::kTcBN, (M + BM - 1) / BM);
   if (grid.y > 65535) return BL_ERR_UNSUPPORTED;
-  kern<<<grid, 192, Cfg::kSmem, st>>>(tm_x, tm_w, eta, gamma, M, K, N, y, y_int);
-  return launch_status();
+  return launch_pdl(kern, grid, dim3(192), Cfg::kSmem, st, tm_x, tm_w, eta, gamma, M, K, N, y, y_int);
 }
 
 template <typename OutT>
@@ -210,35 +221,40 @@ bool fast_layout_ok(int64_t K, const void* xq, const void* packed, const void* y
 bl_path select_path(int64_t M, int64_t K, const void* xq, const void* packed, const void* y,
                     const void* y_int) {
   if (!fast_layout_ok(K, xq, packed, y, y_int) || K > (1 << 30)) return BL_PATH_GENERIC;
-  if (M <= kGemvAutoMaxM && static_cast<int64_t>(M) * K <= kGemvMaxSmem) return BL_PATH_GEMV;
+  if (M <= kGemvAutoMaxM && static_cast<int64_t>(M) * K <= kGemvMaxXBytes && K <= kGemvMaxK)
+    return BL_PATH_GEMV;
   return BL_PATH_TCGEN05;
 }
 
 bl_status forward_impl(const int8_t* xq, const float* eta, const int32_t* xsum, int64_t M,
                        int64_t K, const uint8_t* packed, const float* gamma, int64_t N, void* y,
-                       bl_dtype ydt, int32_t* y_int, bl_path path, void* stream) {
-  if (!xq || !eta || !xsum || !packed || !gamma || !y) return BL_ERR_INVALID_ARG;
+                       bl_dtype ydt, int32_t* y_int, bl_path path, unsigned flags, void* stream) {
   if (M < 0 || K < 1 || N < 1) return BL_ERR_INVALID_ARG;
   if (ydt != BL_F32 && ydt != BL_BF16) return BL_ERR_INVALID_ARG;
   if (path < BL_PATH_AUTO || path > BL_PATH_GENERIC) return BL_ERR_INVALID_ARG;
+  if (!packed || !gamma) return BL_ERR_INVALID_ARG;
+  if (M == 0) return BL_OK;  // empty batch: the M-sized buffers may be NULL
+  if (!xq || !eta || !xsum || !y) return BL_ERR_INVALID_ARG;
   if (127 * K >= (int64_t{1} << 31)) return BL_ERR_UNSUPPORTED;
   if (!aligned(eta, 4) || !aligned(xsum, 4) || !aligned(gamma, 4) ||
       (y_int && !aligned(y_int, 4)) || !aligned(y, ydt == BL_F32 ? 4 : 2))
     return BL_ERR_ALIGNMENT;
-  if (M == 0) return BL_OK;
   int sms = 148;
   bl_status st = device_info(&sms);
   if (st != BL_OK) return st;
   if (path == BL_PATH_AUTO) path = select_path(M, K, xq, packed, y, y_int);
   const cudaStream_t s = as_stream(stream);
   if (path == BL_PATH_GEMV) {
-    if (!fast_layout_ok(K, xq, packed, y, y_int) || M > kGemvMaxM ||
-        M * K > kGemvMaxSmem || N > INT32_MAX / 2)
+    if (!fast_layout_ok(K, xq, packed, y, y_int) || M > kGemvMaxM || M * K > kGemvMaxXBytes ||
+        K > kGemvMaxK ||
+        N > INT32_MAX / 2)
       return BL_ERR_UNSUPPORTED;
-    return ydt == BL_F32
-               ? launch_gemv<float>(xq, eta, xsum, (int)M, (int)K, packed, gamma, (int)N, y, y_int, sms, s)
-               : launch_gemv<__nv_bfloat16>(xq, eta, xsum, (int)M, (int)K, packed, gamma, (int)N, y,
-                                            y_int, sms, s);
+    bl::DecodeArgs a = {};
+    a.x = xq; a.eta = eta; a.xsum = xsum; a.M = (int)M; a.K = (int)K; a.N = (int)N;
+    a.packed = packed; a.gamma = gamma; a.y = y; a.y_int = y_int;
+    a.weights_static = (flags & BL_FLAG_WEIGHTS_STATIC) ? 1 : 0;
+    return ydt == BL_F32 ? launch_decode<false, int8_t, float>(a, sms, s)
+                         : launch_decode<false, int8_t, __nv_bfloat16>(a, sms, s);
   }
   if (path == BL_PATH_TCGEN05) {
     if (!fast_layout_ok(K, xq, packed, y, y_int) || M > INT32_MAX / 2 || N > INT32_MAX / 2 ||
@@ -308,12 +324,12 @@ bl_status bitlinear_pack_weights(const float* W, int64_t N, int64_t K, uint8_t* 
 
 bl_status bitlinear_quant_act(const void* x, bl_dtype xdt, int64_t M, int64_t K, int8_t* xq,
                               float* eta, int32_t* xsum, void* stream) {
-  if (!x || !xq || !eta || !xsum) return BL_ERR_INVALID_ARG;
   if (M < 0 || K < 1) return BL_ERR_INVALID_ARG;
   if (xdt != BL_F32 && xdt != BL_BF16) return BL_ERR_INVALID_ARG;
+  if (M == 0) return BL_OK;  // empty batch: the buffers may be NULL
+  if (!x || !xq || !eta || !xsum) return BL_ERR_INVALID_ARG;
   if (!aligned(x, xdt == BL_F32 ? 4 : 2) || !aligned(eta, 4) || !aligned(xsum, 4))
     return BL_ERR_ALIGNMENT;
-  if (M == 0) return BL_OK;
   int sms = 148;
   bl_status st = device_info(&sms);
   if (st != BL_OK) return st;
@@ -322,27 +338,64 @@ bl_status bitlinear_quant_act(const void* x, bl_dtype xdt, int64_t M, int64_t K,
   if (ctas > static_cast<int64_t>(sms) * 64) ctas = static_cast<int64_t>(sms) * 64;
   if (xdt == BL_BF16) {
     const int vec = (K % 8 == 0) && aligned(x, 16) && aligned(xq, 8);
-    bl::k_quant_act<__nv_bfloat16><<<static_cast<int>(ctas), 256, 0, s>>>(
-        static_cast<const __nv_bfloat16*>(x), M, K, vec, xq, eta, xsum);
-  } else {
-    const int vec = (K % 4 == 0) && aligned(x, 16) && aligned(xq, 4);
-    bl::k_quant_act<float><<<static_cast<int>(ctas), 256, 0, s>>>(static_cast<const float*>(x), M,
-                                                                   K, vec, xq, eta, xsum);
+    return launch_pdl(bl::k_quant_act<__nv_bfloat16>, dim3(static_cast<unsigned>(ctas)), dim3(256),
+                      0, s, static_cast<const __nv_bfloat16*>(x), M, K, vec, xq, eta, xsum);
   }
-  return launch_status();
+  const int vec = (K % 4 == 0) && aligned(x, 16) && aligned(xq, 4);
+  return launch_pdl(bl::k_quant_act<float>, dim3(static_cast<unsigned>(ctas)), dim3(256), 0, s,
+                    static_cast<const float*>(x), M, K, vec, xq, eta, xsum);
 }
 
 bl_status bitlinear_forward(const int8_t* xq, const float* eta, const int32_t* xsum, int64_t M,
                             int64_t K, const uint8_t* packed, const float* gamma, int64_t N,
                             void* y, bl_dtype ydt, int32_t* y_int, void* stream) {
-  return forward_impl(xq, eta, xsum, M, K, packed, gamma, N, y, ydt, y_int, BL_PATH_AUTO, stream);
+  return forward_impl(xq, eta, xsum, M, K, packed, gamma, N, y, ydt, y_int, BL_PATH_AUTO, 0u, stream);
 }
 
 bl_status bitlinear_forward_path(const int8_t* xq, const float* eta, const int32_t* xsum,
                                  int64_t M, int64_t K, const uint8_t* packed, const float* gamma,
                                  int64_t N, void* y, bl_dtype ydt, int32_t* y_int, bl_path path,
-                                 void* stream) {
-  return forward_impl(xq, eta, xsum, M, K, packed, gamma, N, y, ydt, y_int, path, stream);
+                                 unsigned flags, void* stream) {
+  return forward_impl(xq, eta, xsum, M, K, packed, gamma, N, y, ydt, y_int, path, flags, stream);
+}
+
+bl_status bitlinear_linear(const void* x, bl_dtype xdt, int64_t M, int64_t K, const uint8_t* packed,
+                           const float* gamma, int64_t N, void* y, bl_dtype ydt, int8_t* xq,
+                           float* eta, int32_t* xsum, int32_t* y_int, unsigned flags,
+                           void* stream) {
+  if (M < 0 || K < 1 || N < 1) return BL_ERR_INVALID_ARG;
+  if ((xdt != BL_F32 && xdt != BL_BF16) || (ydt != BL_F32 && ydt != BL_BF16))
+    return BL_ERR_INVALID_ARG;
+  if (!packed || !gamma) return BL_ERR_INVALID_ARG;
+  if (M == 0) return BL_OK;
+  if (!x || !y) return BL_ERR_INVALID_ARG;
+  if (127 * K >= (int64_t{1} << 31)) return BL_ERR_UNSUPPORTED;
+  const bool fused = M <= kGemvAutoMaxM && M * K <= kGemvMaxXBytes && K <= kGemvMaxK && K % 64 == 0 &&
+                     aligned(x, 16) && aligned(packed, 16) && aligned(y, 16) &&
+                     (!y_int || aligned(y_int, 16)) && (!xq || aligned(xq, 16)) &&
+                     (!eta || aligned(eta, 4)) && (!xsum || aligned(xsum, 4)) && N <= INT32_MAX / 2;
+  if (!fused) {
+    // Two kernels: quantise into the caller's x~ buffers, then accumulate.
+    if (!xq || !eta || !xsum) return BL_ERR_INVALID_ARG;
+    bl_status st = bitlinear_quant_act(x, xdt, M, K, xq, eta, xsum, stream);
+    if (st != BL_OK) return st;
+    return forward_impl(xq, eta, xsum, M, K, packed, gamma, N, y, ydt, y_int, BL_PATH_AUTO, flags,
+                        stream);
+  }
+  int sms = 148;
+  bl_status st = device_info(&sms);
+  if (st != BL_OK) return st;
+  bl::DecodeArgs a = {};
+  a.x = x; a.M = (int)M; a.K = (int)K; a.N = (int)N;
+  a.packed = packed; a.gamma = gamma; a.y = y; a.y_int = y_int;
+  a.weights_static = (flags & BL_FLAG_WEIGHTS_STATIC) ? 1 : 0;
+  a.xq_out = xq; a.eta_out = eta; a.xsum_out = xsum;
+  const cudaStream_t s = as_stream(stream);
+  if (xdt == BL_BF16)
+    return ydt == BL_F32 ? launch_decode<true, __nv_bfloat16, float>(a, sms, s)
+                         : launch_decode<true, __nv_bfloat16, __nv_bfloat16>(a, sms, s);
+  return ydt == BL_F32 ? launch_decode<true, float, float>(a, sms, s)
+                       : launch_decode<true, float, __nv_bfloat16>(a, sms, s);
 }
 
 bl_path bitlinear_select_path(int64_t M, int64_t K, int64_t N, const void* xq, const void* packed,

@@ -252,4 +252,15 @@ __device__ __forceinline__ float rescale(int32_t y_int, float s) {
   return __fmul_rn(__int2float_rn(y_int), s);
 }
 
+template <typename OutT>
+__device__ __forceinline__ void store_out(void* y, int64_t idx, float v);
+template <>
+__device__ __forceinline__ void store_out<float>(void* y, int64_t idx, float v) {
+  static_cast<float*>(y)[idx] = v;
+}
+template <>
+__device__ __forceinline__ void store_out<__nv_bfloat16>(void* y, int64_t idx, float v) {
+  static_cast<__nv_bfloat16*>(y)[idx] = __float2bfloat16_rn(v);
+}
+
 }  // namespace bl

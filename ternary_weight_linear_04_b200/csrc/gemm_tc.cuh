@@ -26,7 +26,6 @@
 #include <cuda.h>
 
 #include "common.cuh"
-#include "gemv.cuh"
 
 namespace bl {
 
@@ -88,6 +87,8 @@ __global__ void __launch_bounds__(192, 1)
     tmem_alloc(tmem_slot, Cfg::kTmemCols);
     tmem_relinquish();
   }
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   {
     const float gamma = *gamma_p;
     for (int i = threadIdx.x; i < BM; i += blockDim.x)

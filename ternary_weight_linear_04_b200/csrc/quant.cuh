@@ -23,8 +23,19 @@ __device__ __forceinline__ float load_as_f32<__nv_bfloat16>(const __nv_bfloat16*
   return __bfloat162float(*p);
 }
 
-__device__ __forceinline__ int32_t quantise_one(float x, float eta) {
-  const float q = __fdiv_rn(__fmul_rn(x, 127.0f), eta);
+// x~ = clip(RNE(RN32(RN32(x * 127) / eta)), -127, 127), computed exactly but
+// without a division per element.  Only the integer RNE(q) is needed, and it
+// only depends on which side of the nearest half-integer q falls.  With
+// rcp = RN32(1/eta) the product q' = RN32(a * rcp) is within 2^-23 * |a/eta|
+// <= 1.6e-5 of a/eta, and q = RN32(a/eta) within 3.9e-6 of it (|a/eta| <=
+// 127), so |q - q'| < 2e-5.  If q' is farther than 2^-14 (6.1e-5) from its
+// nearest half-integer, q lies strictly on the same side and RNE(q) =
+// RNE(q'); otherwise the IEEE quotient itself is formed.
+__device__ __forceinline__ int32_t quantise_fast(float x, float eta, float rcp) {
+  const float a = __fmul_rn(x, 127.0f);
+  float q = __fmul_rn(a, rcp);
+  const float fr = q - floorf(q);
+  if (fabsf(fr - 0.5f) < 6.103515625e-05f) q = __fdiv_rn(a, eta);
   const float r = fminf(fmaxf(rintf(q), -127.0f), 127.0f);  // rintf: nearest, ties to even
   return static_cast<int32_t>(r);
 }
@@ -102,6 +113,8 @@ __global__ void __launch_bounds__(256) k_quant_act(const T* __restrict__ x, int6
   __shared__ float redf[8];
   __shared__ int32_t redi[8];
   constexpr int V = QVec<T>::kN;
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   for (int64_t m = blockIdx.x; m < M; m += gridDim.x) {
     const T* row = x + m * K;
     int8_t* qrow = xq + m * K;
@@ -118,6 +131,7 @@ __global__ void __launch_bounds__(256) k_quant_act(const T* __restrict__ x, int6
     }
     amax = block_max_256(amax, redf);
     const float eta = fmaxf(amax, 1e-5f);
+    const float rcp = __frcp_rn(eta);
     int32_t sum = 0;
     if (vec) {
       for (int64_t k = static_cast<int64_t>(threadIdx.x) * V; k < K; k += 256 * V) {
@@ -126,14 +140,14 @@ __global__ void __launch_bounds__(256) k_quant_act(const T* __restrict__ x, int6
         int32_t q[V];
 #pragma unroll
         for (int i = 0; i < V; ++i) {
-          q[i] = quantise_one(f[i], eta);
+          q[i] = quantise_fast(f[i], eta, rcp);
           sum += q[i];
         }
         QVec<T>::store(qrow + k, q);
       }
     } else {
       for (int64_t k = threadIdx.x; k < K; k += 256) {
-        const int32_t q = quantise_one(load_as_f32(row + k), eta);
+        const int32_t q = quantise_fast(load_as_f32(row + k), eta, rcp);
         sum += q;
         qrow[k] = static_cast<int8_t>(q);
       }

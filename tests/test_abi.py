@@ -55,6 +55,7 @@ def test_bad_arguments_are_rejected_without_a_launch(L):
     assert L.bitlinear_pack_weights(fake, 1 << 21, 1 << 20, fake, fake, fake, None) == _lib.BL_ERR_UNSUPPORTED
     assert L.bitlinear_pack_weights(P(258), 4, 4, fake, fake, fake, None) == _lib.BL_ERR_ALIGNMENT
     assert L.bitlinear_quant_act(None, 0, 1, 4, fake, fake, fake, None) == _lib.BL_ERR_INVALID_ARG
+    assert L.bitlinear_quant_act(None, 0, 0, 4, None, None, None, None) == _lib.BL_OK
     assert L.bitlinear_quant_act(fake, 7, 1, 4, fake, fake, fake, None) == _lib.BL_ERR_INVALID_ARG
     assert L.bitlinear_quant_act(fake, 0, -1, 4, fake, fake, fake, None) == _lib.BL_ERR_INVALID_ARG
     assert L.bitlinear_quant_act(fake, 0, 1, 0, fake, fake, fake, None) == _lib.BL_ERR_INVALID_ARG
@@ -68,8 +69,16 @@ def test_bad_arguments_are_rejected_without_a_launch(L):
     assert fwd(fake, fake, fake, 1, 1 << 25, fake, fake, 8, fake, 0, None, None) == _lib.BL_ERR_UNSUPPORTED
     assert fwd(fake, P(258), fake, 1, 64, fake, fake, 8, fake, 0, None, None) == _lib.BL_ERR_ALIGNMENT
     assert fwd(fake, fake, fake, 0, 64, fake, fake, 8, fake, 0, None, None) == _lib.BL_OK
-    assert L.bitlinear_forward_path(fake, fake, fake, 1, 64, fake, fake, 8, fake, 0, None, 9,
+    assert fwd(None, None, None, 0, 64, fake, fake, 8, None, 0, None, None) == _lib.BL_OK
+    assert fwd(None, None, None, 0, 64, None, fake, 8, None, 0, None, None) == _lib.BL_ERR_INVALID_ARG
+    assert L.bitlinear_forward_path(fake, fake, fake, 1, 64, fake, fake, 8, fake, 0, None, 9, 0,
                                     None) == _lib.BL_ERR_INVALID_ARG
+    lin = L.bitlinear_linear
+    assert lin(fake, 0, 1, 64, None, fake, 8, fake, 0, None, None, None, None, 0, None) == _lib.BL_ERR_INVALID_ARG
+    assert lin(fake, 3, 1, 64, fake, fake, 8, fake, 0, None, None, None, None, 0, None) == _lib.BL_ERR_INVALID_ARG
+    assert lin(None, 0, 0, 64, fake, fake, 8, None, 0, None, None, None, None, 0, None) == _lib.BL_OK
+    # a prefill-sized batch needs the caller's x~ scratch
+    assert lin(fake, 1, 64, 64, fake, fake, 8, fake, 1, None, None, None, None, 0, None) == _lib.BL_ERR_INVALID_ARG
     assert L.bitlinear_device_error(None, None) == _lib.BL_ERR_INVALID_ARG
 
 

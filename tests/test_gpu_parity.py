@@ -252,3 +252,78 @@ def test_full_outlier_sweep():
     w = inputs.WORKLOADS["outlier_sweep"]
     W, x = inputs.make_matrix_inputs(w, 0)
     check_full(W, x, w.batches)
+
+
+# ----------------------------------------------------------------- fused per-token layer
+
+@pytest.mark.parametrize("M", [1, 2, 3, 4])
+@pytest.mark.parametrize("K,N", [(64, 5), (3200, 1000), (8640, 333), (28672, 130)])
+@pytest.mark.parametrize("static", [False, True])
+def test_linear_fused_matches_oracle(M, K, N, static):
+    W, x = inputs.make_case(5000 + M + K + N, M, K, N, x_dist="student_t_outliers", act_dtype="bf16")
+    ref_packed, ref_gamma, _ = orc.pack_weights(W)
+    _, _, packed, gamma = gpu_pack(W)
+    torch.cuda.synchronize()
+    xd = torch.from_numpy(x).cuda().to(torch.bfloat16)
+    y, (xq, eta, xsum), y_int = bl.linear(xd, packed, gamma, N, out_dtype=torch.bfloat16,
+                                          want_quant=True, want_int=True, weights_static=static)
+    ref_xq, ref_eta, ref_xsum = orc.quant_act(x)
+    ref_yint, ref_y = orc.forward(ref_xq, ref_eta, ref_packed, ref_gamma, K, N)
+    np.testing.assert_array_equal(xq.cpu().numpy(), ref_xq)
+    np.testing.assert_array_equal(eta.cpu().numpy(), ref_eta)
+    np.testing.assert_array_equal(xsum.cpu().numpy(), ref_xsum)
+    np.testing.assert_array_equal(y_int.cpu().numpy(), ref_yint)
+    np.testing.assert_array_equal(y_bits(y.cpu()), orc.f32_to_bf16_bits(ref_y))
+    y2 = bl.linear(xd, packed, gamma, N, out_dtype=torch.float32)  # no optional outputs
+    np.testing.assert_array_equal(y2.cpu().numpy().view(np.uint32), ref_y.view(np.uint32))
+
+
+@pytest.mark.parametrize("act", ["f32", "bf16"])
+def test_linear_two_kernel_path(act):
+    """M above the decode range: quantise into caller scratch, then tcgen05."""
+    W, x = inputs.make_case(6000, 37, 1024, 300, act_dtype=act)
+    ref_packed, ref_gamma, _ = orc.pack_weights(W)
+    _, _, packed, gamma = gpu_pack(W)
+    y, (xq, eta, xsum) = bl.linear(torch.from_numpy(x).cuda().to(DT[act]), packed, gamma, 300,
+                                   out_dtype=torch.float32, want_quant=True)
+    ref_xq, ref_eta, _ = orc.quant_act(x)
+    _, ref_y = orc.forward(ref_xq, ref_eta, ref_packed, ref_gamma, 1024, 300)
+    np.testing.assert_array_equal(xq.cpu().numpy(), ref_xq)
+    np.testing.assert_array_equal(y.cpu().numpy().view(np.uint32), ref_y.view(np.uint32))
+
+
+def test_chained_layers_under_dependent_launch():
+    """Layer 2 reads layer 1's output.  Launched back to back on one stream
+    with static weights, the second kernel may start streaming its weights
+    early but must read its activations only after the first has finished;
+    a 20-deep chain checks that on every link."""
+    rng = np.random.default_rng(99)
+    K = 1024
+    Ws = [inputs.draw_weights(rng, K, K) for _ in range(4)]
+    packs = [gpu_pack(W)[2:] for W in Ws]
+    ref = [orc.pack_weights(W)[:2] for W in Ws]
+    torch.cuda.synchronize()
+    x = inputs.draw_activations(rng, 1, K, "normal", "bf16")
+    h = torch.from_numpy(x).cuda().to(torch.bfloat16)
+    h_ref = x
+    for i in range(20):
+        pk, g = packs[i % 4]
+        h = bl.linear(h, pk, g, K, out_dtype=torch.bfloat16, weights_static=True)
+        rp, rg = ref[i % 4]
+        xq, eta, _ = orc.quant_act(h_ref)
+        _, y = orc.forward(xq, eta, rp, rg, K, K)
+        h_ref = orc.f32_to_bf16_bits(y).astype(np.uint32) << 16
+        h_ref = h_ref.view(np.float32)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(h.cpu().float().numpy().view(np.uint32), h_ref.view(np.uint32))
+
+
+def test_bitlinear_module():
+    W, x = inputs.make_case(7, 2, 512, 96, act_dtype="bf16")
+    layer = bl.BitLinear.from_latent(torch.from_numpy(W).cuda())
+    torch.cuda.synchronize()
+    y = layer(torch.from_numpy(x).cuda().to(torch.bfloat16))
+    ref_packed, ref_gamma, _ = orc.pack_weights(W)
+    ref_xq, ref_eta, _ = orc.quant_act(x)
+    _, ref_y = orc.forward(ref_xq, ref_eta, ref_packed, ref_gamma, 512, 96)
+    np.testing.assert_array_equal(y_bits(y.cpu()), orc.f32_to_bf16_bits(ref_y))
