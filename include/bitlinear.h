@@ -166,8 +166,9 @@ bl_status bitlinear_forward(const int8_t* xq, const float* eta, const int32_t* x
  * bitlinear_forward with the accumulate kernel and flags chosen by the
  * caller.  BL_PATH_GEMV and BL_PATH_TCGEN05 return BL_ERR_UNSUPPORTED when
  * the inputs do not meet their layout needs (K % 64 == 0, 16-byte
- * alignment; for BL_PATH_GEMV also M <= 8, K <= 65536 and M*K <= 147456); the results of
- * every path are identical.  flags: 0 or BL_FLAG_WEIGHTS_STATIC.
+ * alignment; for BL_PATH_GEMV also M <= 4 and K * M' <= 32768, M' = M
+ * rounded up to 1, 2 or 4); the results of every path are identical.
+ * flags: 0 or BL_FLAG_WEIGHTS_STATIC.
  */
 bl_status bitlinear_forward_path(const int8_t* xq, const float* eta, const int32_t* xsum,
                                  int64_t M, int64_t K,
@@ -187,10 +188,11 @@ bl_status bitlinear_forward_path(const int8_t* xq, const float* eta, const int32
  *   y, ydt, y_int     out  as for bitlinear_forward (y_int optional).
  *   xq, eta, xsum     out  the quantised activations (M x K int8, M fp32,
  *                          M int32).  For decode batches (M <= 4, K % 64 ==
- *                          0, 16-byte aligned x, packed, y) one fused kernel
- *                          runs and these are optional (NULL = not written).
- *                          Otherwise two kernels run and they are required
- *                          scratch (BL_ERR_INVALID_ARG if NULL).
+ *                          0, K * M' <= 32768 with M' = M rounded up to 1,
+ *                          2 or 4, 16-byte aligned x, packed, y) one fused
+ *                          kernel runs and these are optional (NULL = not
+ *                          written).  Otherwise two kernels run and they are
+ *                          required scratch (BL_ERR_INVALID_ARG if NULL).
  *   flags             in   0 or BL_FLAG_WEIGHTS_STATIC.
  */
 bl_status bitlinear_linear(const void* x, bl_dtype xdt, int64_t M, int64_t K,

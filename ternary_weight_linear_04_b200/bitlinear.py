@@ -94,6 +94,13 @@ def forward(xq, eta, xsum, packed, gamma, N, out_dtype=torch.bfloat16, want_int=
     return (y, y_int) if want_int else y
 
 
+def fused_decode_ok(M, K):
+    """Whether bitlinear_linear runs its single fused decode kernel for (M, K)
+    (the same rule as the library; otherwise it needs x~ scratch)."""
+    mt = 1 if M <= 1 else (2 if M <= 2 else 4)
+    return 1 <= M <= 4 and K % 64 == 0 and K * mt <= 32768
+
+
 def linear(x, packed, gamma, N, out_dtype=torch.bfloat16, want_quant=False, want_int=False,
            weights_static=False, stream=None, out=None, scratch=None):
     """The whole per-token layer (quantise + accumulate + rescale) in one call.
@@ -106,7 +113,7 @@ def linear(x, packed, gamma, N, out_dtype=torch.bfloat16, want_quant=False, want
         raise ValueError("packed shape %s does not match N=%d, K=%d" % (tuple(packed.shape), N, K))
     dev = x.device
     y = out if out is not None else torch.empty((M, N), dtype=out_dtype, device=dev)
-    decode = M <= 4 and K % 64 == 0
+    decode = fused_decode_ok(M, K)
     if scratch is not None:
         xq, eta, xsum = scratch
     elif want_quant or not decode:

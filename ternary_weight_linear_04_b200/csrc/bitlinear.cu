@@ -23,10 +23,17 @@
 namespace {
 
 constexpr int kMaxDevices = 64;
-constexpr int kGemvMaxM = 8;          // largest token count the CUDA-core decode kernel takes
-constexpr int kGemvAutoMaxM = 4;      // auto dispatch: above this, tensor cores
-constexpr int64_t kGemvMaxXBytes = 144 * 1024;  // M*K activation bytes the decode kernel stages
-constexpr int64_t kGemvMaxK = 4 * bl::kDecStageBytes;      // a stage holds at least one packed row
+constexpr int kGemvMaxM = 4;  // largest token count the CUDA-core decode kernel takes
+
+// Tokens rounded up to the decode kernel's widths (1, 2, 4).
+inline int decode_mt(int64_t M) { return M <= 1 ? 1 : (M <= 2 ? 2 : 4); }
+
+// Whether the decode kernel takes (M, K): K % 64 == 0, M <= 4 and
+// K * MT <= 32768 (each thread stages at most 8 words x MT tokens of
+// activations, 32 KB of shared memory per CTA).
+inline bool decode_ok(int64_t M, int64_t K) {
+  return M >= 1 && M <= kGemvMaxM && K % 64 == 0 && K * decode_mt(M) <= 32768;
+}
 
 inline bool aligned(const void* p, uintptr_t a) {
   return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0;
@@ -91,17 +98,24 @@ bl_status device_info(int* sms) {
   return d.ok ? BL_OK : BL_ERR_UNSUPPORTED;
 }
 
-// Raise a kernel's dynamic shared memory limit once per device.
+// Once per device and kernel: raise the dynamic shared memory limit and ask
+// for the largest shared-memory carveout.  Every kernel of the library uses
+// the same carveout, so CTAs of consecutive kernels can share an SM (the
+// carveout of an SM only changes while it is idle), which is what lets a
+// kernel launched with programmatic dependent launch start early.
 template <typename Kern>
 bool ensure_smem(Kern kern, size_t bytes, int* done_flags) {
-  if (bytes <= 48 * 1024) return true;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
-  if (done_flags[dev] >= static_cast<int>(bytes)) return true;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (done_flags[dev] >= static_cast<int>(bytes) && done_flags[dev] > 0) return true;
+  if (bytes > 48 * 1024 &&
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(bytes)) != cudaSuccess)
     return false;
-  done_flags[dev] = static_cast<int>(bytes);
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           cudaSharedmemCarveoutMaxShared) != cudaSuccess)
+    return false;
+  done_flags[dev] = bytes > 0 ? static_cast<int>(bytes) : 1;
   return true;
 }
 
@@ -140,29 +154,51 @@ bool make_tmap_u8(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t col
 
 // ------------------------------------------------------------ launchers
 
-// Decode kernel (M <= 8 tokens): one CTA per SM-slot, each owning a
-// contiguous block of rows.  FUSED = quantise x inside the kernel.
-template <int MT, bool FUSED, typename XT, typename OutT>
-bl_status launch_decode_mt(const bl::DecodeArgs& a, int sms, cudaStream_t st) {
+// Decode kernel (M <= 4 tokens): one CTA per SM, each owning a contiguous
+// block of rows, so the next kernel's CTA fits beside it under programmatic
+// dependent launch.  XT = activation type when the quantiser is fused, or
+// bl::DecNoFuse when x~ is given.
+template <int MT, typename XT, typename OutT>
+bl_status launch_decode_kernel(const bl::DecodeArgs& a0, int sms, cudaStream_t st) {
   static int smem_done[kMaxDevices] = {0};
-  const size_t smem = bl::DecSmem<MT>::bytes(a.K);
-  auto kern = bl::k_decode<MT, FUSED, XT, OutT>;
-  if (!ensure_smem(kern, smem, smem_done)) return BL_ERR_CUDA;
-  int64_t grid = static_cast<int64_t>(sms) * bl::DecOcc<MT>::kCtasPerSm;
-  const int64_t max_ctas = (static_cast<int64_t>(a.N) + 3) / 4;
-  if (grid > max_ctas) grid = max_ctas;
-  bl::DecodeArgs args = a;
-  args.rows_per_cta = static_cast<int>((a.N + grid - 1) / grid);
-  grid = (a.N + args.rows_per_cta - 1) / args.rows_per_cta;
-  return launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(bl::kDecThreads), smem, st, args);
+  bl::DecodeArgs a = a0;
+  const int64_t P = a.K / 4;
+  const int64_t nwj = (a.K / 16 + bl::kDecColThreads - 1) / bl::kDecColThreads;
+  int64_t rps = bl::kDecStageTarget / P;  // rows per stage (one chunk)
+  if (rps > 32 / MT) rps = 32 / MT;
+  if (rps < 1) rps = 1;
+  // One CTA per SM, unless that would give a CTA more chunks than its
+  // reduction slots hold.
+  int64_t grid = sms;
+  const int64_t min_grid = (a.N + rps * bl::kDecMaxChunks - 1) / (rps * bl::kDecMaxChunks);
+  if (grid < min_grid) grid = min_grid;
+  if (grid > a.N) grid = a.N;
+  a.rows_per_cta = static_cast<int>((a.N + grid - 1) / grid);
+  grid = (a.N + a.rows_per_cta - 1) / a.rows_per_cta;
+  if (rps > a.rows_per_cta) rps = a.rows_per_cta;
+  a.rows_per_stage = static_cast<int>(rps);
+  const int64_t chunks = (a.rows_per_cta + rps - 1) / rps;
+  if (chunks > bl::kDecMaxChunks || grid > 0x7FFFFFFF) return BL_ERR_UNSUPPORTED;
+  int64_t stages = bl::kDecSmemBudget / (rps * P);
+  if (stages > bl::kDecMaxStages) stages = bl::kDecMaxStages;
+  if (stages > chunks) stages = chunks;
+  if (stages < 1) stages = 1;
+  a.stages = static_cast<int>(stages);
+  const size_t smem = static_cast<size_t>(nwj * MT * bl::kDecColThreads * 16) +
+                      static_cast<size_t>(stages * rps * P) + sizeof(bl::DecTail);
+  auto kern = bl::k_decode<MT, XT, OutT>;
+  if (!ensure_smem(kern, 227 * 1024, smem_done)) return BL_ERR_CUDA;
+  return launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(bl::kDecThreads), smem, st, a);
 }
 
-template <bool FUSED, typename XT, typename OutT>
+template <typename XT, typename OutT>
 bl_status launch_decode(const bl::DecodeArgs& a, int sms, cudaStream_t st) {
-  if (a.M <= 1) return launch_decode_mt<1, FUSED, XT, OutT>(a, sms, st);
-  if (a.M <= 2) return launch_decode_mt<2, FUSED, XT, OutT>(a, sms, st);
-  if (a.M <= 4) return launch_decode_mt<4, FUSED, XT, OutT>(a, sms, st);
-  return launch_decode_mt<8, FUSED, XT, OutT>(a, sms, st);
+  if (!decode_ok(a.M, a.K)) return BL_ERR_UNSUPPORTED;
+  switch (decode_mt(a.M)) {
+    case 1: return launch_decode_kernel<1, XT, OutT>(a, sms, st);
+    case 2: return launch_decode_kernel<2, XT, OutT>(a, sms, st);
+    default: return launch_decode_kernel<4, XT, OutT>(a, sms, st);
+  }
 }
 
 template <typename OutT>
@@ -176,6 +212,8 @@ bl_status launch_generic(const int8_t* xq, const float* eta, int64_t M, int64_t 
     if (ctas > static_cast<int64_t>(sms) * 16) ctas = static_cast<int64_t>(sms) * 16;
     dim3 grid(static_cast<unsigned>(ctas), static_cast<unsigned>(mb));
     const int64_t m_off = mb0 * 8;
+    static int carve_done[kMaxDevices] = {0};
+    if (!ensure_smem(bl::k_gemv_generic<OutT>, 0, carve_done)) return BL_ERR_CUDA;
     const bl_status s = launch_pdl(
         bl::k_gemv_generic<OutT>, grid, dim3(256), 0, st, xq + m_off * K, eta + m_off, M - m_off,
         K, packed, gamma, N, static_cast<void*>(static_cast<char*>(y) + m_off * N * sizeof(OutT)),
@@ -221,8 +259,7 @@ bool fast_layout_ok(int64_t K, const void* xq, const void* packed, const void* y
 bl_path select_path(int64_t M, int64_t K, const void* xq, const void* packed, const void* y,
                     const void* y_int) {
   if (!fast_layout_ok(K, xq, packed, y, y_int) || K > (1 << 30)) return BL_PATH_GENERIC;
-  if (M <= kGemvAutoMaxM && static_cast<int64_t>(M) * K <= kGemvMaxXBytes && K <= kGemvMaxK)
-    return BL_PATH_GEMV;
+  if (decode_ok(M, K)) return BL_PATH_GEMV;
   return BL_PATH_TCGEN05;
 }
 
@@ -245,16 +282,15 @@ bl_status forward_impl(const int8_t* xq, const float* eta, const int32_t* xsum, 
   if (path == BL_PATH_AUTO) path = select_path(M, K, xq, packed, y, y_int);
   const cudaStream_t s = as_stream(stream);
   if (path == BL_PATH_GEMV) {
-    if (!fast_layout_ok(K, xq, packed, y, y_int) || M > kGemvMaxM || M * K > kGemvMaxXBytes ||
-        K > kGemvMaxK ||
+    if (!fast_layout_ok(K, xq, packed, y, y_int) || !decode_ok(M, K) ||
         N > INT32_MAX / 2)
       return BL_ERR_UNSUPPORTED;
     bl::DecodeArgs a = {};
     a.x = xq; a.eta = eta; a.xsum = xsum; a.M = (int)M; a.K = (int)K; a.N = (int)N;
     a.packed = packed; a.gamma = gamma; a.y = y; a.y_int = y_int;
     a.weights_static = (flags & BL_FLAG_WEIGHTS_STATIC) ? 1 : 0;
-    return ydt == BL_F32 ? launch_decode<false, int8_t, float>(a, sms, s)
-                         : launch_decode<false, int8_t, __nv_bfloat16>(a, sms, s);
+    return ydt == BL_F32 ? launch_decode<bl::DecNoFuse, float>(a, sms, s)
+                         : launch_decode<bl::DecNoFuse, __nv_bfloat16>(a, sms, s);
   }
   if (path == BL_PATH_TCGEN05) {
     if (!fast_layout_ok(K, xq, packed, y, y_int) || M > INT32_MAX / 2 || N > INT32_MAX / 2 ||
@@ -338,10 +374,14 @@ bl_status bitlinear_quant_act(const void* x, bl_dtype xdt, int64_t M, int64_t K,
   if (ctas > static_cast<int64_t>(sms) * 64) ctas = static_cast<int64_t>(sms) * 64;
   if (xdt == BL_BF16) {
     const int vec = (K % 8 == 0) && aligned(x, 16) && aligned(xq, 8);
+    static int carve_done[kMaxDevices] = {0};
+    if (!ensure_smem(bl::k_quant_act<__nv_bfloat16>, 0, carve_done)) return BL_ERR_CUDA;
     return launch_pdl(bl::k_quant_act<__nv_bfloat16>, dim3(static_cast<unsigned>(ctas)), dim3(256),
                       0, s, static_cast<const __nv_bfloat16*>(x), M, K, vec, xq, eta, xsum);
   }
   const int vec = (K % 4 == 0) && aligned(x, 16) && aligned(xq, 4);
+  static int carve_done_f[kMaxDevices] = {0};
+  if (!ensure_smem(bl::k_quant_act<float>, 0, carve_done_f)) return BL_ERR_CUDA;
   return launch_pdl(bl::k_quant_act<float>, dim3(static_cast<unsigned>(ctas)), dim3(256), 0, s,
                     static_cast<const float*>(x), M, K, vec, xq, eta, xsum);
 }
@@ -370,7 +410,7 @@ bl_status bitlinear_linear(const void* x, bl_dtype xdt, int64_t M, int64_t K, co
   if (M == 0) return BL_OK;
   if (!x || !y) return BL_ERR_INVALID_ARG;
   if (127 * K >= (int64_t{1} << 31)) return BL_ERR_UNSUPPORTED;
-  const bool fused = M <= kGemvAutoMaxM && M * K <= kGemvMaxXBytes && K <= kGemvMaxK && K % 64 == 0 &&
+  const bool fused = decode_ok(M, K) &&
                      aligned(x, 16) && aligned(packed, 16) && aligned(y, 16) &&
                      (!y_int || aligned(y_int, 16)) && (!xq || aligned(xq, 16)) &&
                      (!eta || aligned(eta, 4)) && (!xsum || aligned(xsum, 4)) && N <= INT32_MAX / 2;
@@ -392,10 +432,10 @@ bl_status bitlinear_linear(const void* x, bl_dtype xdt, int64_t M, int64_t K, co
   a.xq_out = xq; a.eta_out = eta; a.xsum_out = xsum;
   const cudaStream_t s = as_stream(stream);
   if (xdt == BL_BF16)
-    return ydt == BL_F32 ? launch_decode<true, __nv_bfloat16, float>(a, sms, s)
-                         : launch_decode<true, __nv_bfloat16, __nv_bfloat16>(a, sms, s);
-  return ydt == BL_F32 ? launch_decode<true, float, float>(a, sms, s)
-                       : launch_decode<true, float, __nv_bfloat16>(a, sms, s);
+    return ydt == BL_F32 ? launch_decode<__nv_bfloat16, float>(a, sms, s)
+                         : launch_decode<__nv_bfloat16, __nv_bfloat16>(a, sms, s);
+  return ydt == BL_F32 ? launch_decode<float, float>(a, sms, s)
+                       : launch_decode<float, __nv_bfloat16>(a, sms, s);
 }
 
 bl_path bitlinear_select_path(int64_t M, int64_t K, int64_t N, const void* xq, const void* packed,

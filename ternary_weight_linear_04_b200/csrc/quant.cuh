@@ -31,13 +31,43 @@ __device__ __forceinline__ float load_as_f32<__nv_bfloat16>(const __nv_bfloat16*
 // 127), so |q - q'| < 2e-5.  If q' is farther than 2^-14 (6.1e-5) from its
 // nearest half-integer, q lies strictly on the same side and RNE(q) =
 // RNE(q'); otherwise the IEEE quotient itself is formed.
+// The exact quotient, out of line so the common path stays a few instructions
+// and the divide is a real (rarely taken) branch rather than predicated code.
+__device__ __noinline__ float quotient_exact(float a, float eta) { return __fdiv_rn(a, eta); }
+
 __device__ __forceinline__ int32_t quantise_fast(float x, float eta, float rcp) {
   const float a = __fmul_rn(x, 127.0f);
   float q = __fmul_rn(a, rcp);
   const float fr = q - floorf(q);
-  if (fabsf(fr - 0.5f) < 6.103515625e-05f) q = __fdiv_rn(a, eta);
+  if (fabsf(fr - 0.5f) < 6.103515625e-05f) q = quotient_exact(a, eta);
   const float r = fminf(fmaxf(rintf(q), -127.0f), 127.0f);  // rintf: nearest, ties to even
   return static_cast<int32_t>(r);
+}
+
+// The same for 16 values at once, with no branch in the common path: all 16
+// candidates are formed first, and only if some lane of the warp has a value
+// near a tie does the warp take the (rare) exact fix-up loop.
+__device__ __forceinline__ void quantise16(const float (&f)[16], float eta, float rcp,
+                                           int32_t (&q)[16]) {
+  float a[16];
+  uint32_t near = 0;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    a[i] = __fmul_rn(f[i], 127.0f);
+    const float c = __fmul_rn(a[i], rcp);
+    const float fr = c - floorf(c);
+    near |= (fabsf(fr - 0.5f) < 6.103515625e-05f ? 1u : 0u) << i;
+    q[i] = static_cast<int32_t>(fminf(fmaxf(rintf(c), -127.0f), 127.0f));
+  }
+  if (__any_sync(__activemask(), near != 0)) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      if ((near >> i) & 1u) {
+        const float c = quotient_exact(a[i], eta);
+        q[i] = static_cast<int32_t>(fminf(fmaxf(rintf(c), -127.0f), 127.0f));
+      }
+    }
+  }
 }
 
 // Block-wide reductions over 256 threads.

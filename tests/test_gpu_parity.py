@@ -96,6 +96,8 @@ def test_ragged_k_generic(K):
                                    (4, 3200, 1000), (8, 1024, 257)])
 @pytest.mark.parametrize("out", ["f32", "bf16"])
 def test_paths_agree_with_oracle(path, M, K, N, out):
+    if path == "gemv" and M > 4:
+        pytest.skip("the decode kernel takes at most 4 tokens")
     W, x = inputs.make_case(1000 + M * 7 + K + N, M, K, N, act_dtype="bf16")
     check_layer(W, x, "bf16", out, path=path)
 
@@ -257,7 +259,8 @@ def test_full_outlier_sweep():
 # ----------------------------------------------------------------- fused per-token layer
 
 @pytest.mark.parametrize("M", [1, 2, 3, 4])
-@pytest.mark.parametrize("K,N", [(64, 5), (3200, 1000), (8640, 333), (28672, 130)])
+@pytest.mark.parametrize("K,N", [(64, 5), (3200, 1000), (4096, 700), (8640, 333), (16384, 77),
+                                 (28672, 130)])
 @pytest.mark.parametrize("static", [False, True])
 def test_linear_fused_matches_oracle(M, K, N, static):
     W, x = inputs.make_case(5000 + M + K + N, M, K, N, x_dist="student_t_outliers", act_dtype="bf16")
@@ -327,3 +330,14 @@ def test_bitlinear_module():
     ref_xq, ref_eta, _ = orc.quant_act(x)
     _, ref_y = orc.forward(ref_xq, ref_eta, ref_packed, ref_gamma, 512, 96)
     np.testing.assert_array_equal(y_bits(y.cpu()), orc.f32_to_bf16_bits(ref_y))
+
+
+@pytest.mark.parametrize("M", [1, 2, 3, 4])
+@pytest.mark.parametrize("K", [64, 4096, 4160, 8192, 12288, 16384, 32768])
+def test_decode_word_widths(M, K):
+    """Every words-per-thread width (1, 2, 4, 8) and stage/row-block shape of
+    the decode kernel, with N not a multiple of the rows per CTA."""
+    if K * (1 if M == 1 else (2 if M == 2 else 4)) > 32768:
+        pytest.skip("outside the decode kernel's register budget")
+    W, x = inputs.make_case(9000 + M + K, M, K, 1237, act_dtype="bf16")
+    check_layer(W, x, "bf16", "bf16", path="gemv")
