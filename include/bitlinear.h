@@ -107,6 +107,32 @@ bl_status bitlinear_pack_weights(const float* W, int64_t N, int64_t K,
                                  void* workspace, void* stream);
 
 /*
+ * bitlinear_pack_weights for callers that cannot allocate device memory:
+ * for example a library running inside a host framework that owns every
+ * byte of device memory through its own pool, or a latency-critical path
+ * that must not call cudaMalloc (which can synchronise the device).  The
+ * pages have no counterpart; this is a property of the library, not of the
+ * method.
+ *
+ * Same arguments, results and errors as bitlinear_pack_weights, minus the
+ * workspace: the 2048-byte bucket scratch is a file-scope device array of
+ * the library (256 x 64-bit), held on every GPU that loads the library until
+ * the process exits.  The call allocates nothing (no cudaMalloc, cudaFree
+ * or allocating library routine).
+ *   - Limit: N*K < 2^40 (the exact sum's 64-bit buckets); larger sizes return
+ *     BL_ERR_UNSUPPORTED before anything is launched.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current) and caches it; make
+ *     that first call before any stream capture on the device.
+ *   - Every call on a device shares the one array and clears it first.  Calls
+ *     that may overlap on the GPU (other streams, or other threads' streams,
+ *     without ordering between them) race on it and give wrong gamma values;
+ *     order them, or use bitlinear_pack_weights with separate workspaces.
+ */
+bl_status bitlinear_pack_weights_noalloc(const float* W, int64_t N, int64_t K,
+                                         uint8_t* packed, float* gamma, void* stream);
+
+/*
  * Per-token absmax int8 quantisation of activations.
  * [Production] "2. Absmax Dynamic Activation Quantization" and
  * ActivationQuantizerSTE: eta per token (last dimension), clamp at 1e-5,

@@ -358,6 +358,75 @@ bl_status bitlinear_pack_weights(const float* W, int64_t N, int64_t K, uint8_t* 
   return launch_status();
 }
 
+}  // extern "C"
+
+// ------------------------------------------------------------ allocation-free packing
+//
+// Scratch for bitlinear_pack_weights_noalloc: the 256 exponent buckets of
+// the exact |W| sum (2048 bytes), in a file-scope device array instead of a
+// caller buffer.  Every GPU that loads the library holds one copy until the
+// process exits.  In host code the array's name is only a host-side stand-in
+// for the symbol, so its device address is looked up with
+// cudaGetSymbolAddress, once per device, with that device current.
+namespace {
+
+static __device__ __align__(256) unsigned long long g_pack_scratch[bl::kBuckets];
+
+unsigned long long* g_pack_scratch_ptr[kMaxDevices] = {nullptr};
+std::mutex g_pack_scratch_mu;
+
+bl_status pack_scratch_address(unsigned long long** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return BL_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_pack_scratch_mu);
+  if (!g_pack_scratch_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_pack_scratch) != cudaSuccess || p == nullptr) {
+      (void)cudaGetLastError();
+      return BL_ERR_CUDA;
+    }
+    g_pack_scratch_ptr[dev] = static_cast<unsigned long long*>(p);
+  }
+  *out = g_pack_scratch_ptr[dev];
+  return BL_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+bl_status bitlinear_pack_weights_noalloc(const float* W, int64_t N, int64_t K, uint8_t* packed,
+                                         float* gamma, void* stream) {
+  if (!W || !packed || !gamma) return BL_ERR_INVALID_ARG;
+  if (N < 1 || K < 1) return BL_ERR_INVALID_ARG;
+  // The fixed 2048-byte scratch holds 64-bit bucket sums of 24-bit
+  // mantissas: exact for fewer than 2^40 weights.
+  if (N > (int64_t{1} << 40) / K) return BL_ERR_UNSUPPORTED;
+  if (!aligned(W, 4) || !aligned(gamma, 4)) return BL_ERR_ALIGNMENT;
+  int sms = 148;
+  bl_status st = device_info(&sms);
+  if (st != BL_OK) return st;
+  unsigned long long* buckets = nullptr;
+  if ((st = pack_scratch_address(&buckets)) != BL_OK) return st;
+  const cudaStream_t s = as_stream(stream);
+  // The shared array keeps the previous call's sums: clear it first.
+  bl::k_zero_u64<<<1, 256, 0, s>>>(buckets, bl::kBuckets);
+  if ((st = launch_status()) != BL_OK) return st;
+  const int64_t count = N * K;
+  int64_t ctas = (count / 4 + 255) / 256;
+  if (ctas > static_cast<int64_t>(sms) * 8) ctas = static_cast<int64_t>(sms) * 8;
+  if (ctas < 1) ctas = 1;
+  bl::k_absmean_buckets<<<static_cast<int>(ctas), 256, 0, s>>>(W, count, buckets);
+  if ((st = launch_status()) != BL_OK) return st;
+  bl::k_gamma_finalize<<<1, 32, 0, s>>>(buckets, count, gamma);
+  if ((st = launch_status()) != BL_OK) return st;
+  const int64_t bytes = N * ((K + 3) / 4);
+  int64_t pctas = (bytes + 255) / 256;
+  if (pctas > static_cast<int64_t>(sms) * 32) pctas = static_cast<int64_t>(sms) * 32;
+  bl::k_ternarise_pack2<<<static_cast<int>(pctas), 256, 0, s>>>(W, N, K, gamma, packed);
+  return launch_status();
+}
+
 bl_status bitlinear_quant_act(const void* x, bl_dtype xdt, int64_t M, int64_t K, int8_t* xq,
                               float* eta, int32_t* xsum, void* stream) {
   if (M < 0 || K < 1) return BL_ERR_INVALID_ARG;
