@@ -291,9 +291,14 @@ def run_ours(args, world, rank, local):
            "roofline": roofline, "gpu_launches": launches,
            "clocks": clk.summary()}
 
-    if not args.quick:
+    sections = set(args.sections.split(",")) if args.sections else {"e2e", "prefill", "pack"}
+    if args.quick:
+        sections = set()
+    if "e2e" in sections:
         out["e2e"] = run_e2e(args, mats, M, stream, world)
+    if "prefill" in sections:
         out["prefill"] = run_prefill(args, dev, stream, peaks, peak_src, world)
+    if "pack" in sections:
         out["pack"] = run_pack(mats, stream, world)
     if (rank == 0) and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = run_cpu_baseline(args.cpu_seconds)
@@ -511,6 +516,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--m", type=int, default=1, help="tokens per step (decode batch)")
     ap.add_argument("--quick", action="store_true", help="headline only (no e2e/prefill/pack)")
+    ap.add_argument("--sections", default="", help="comma list of extra sections: e2e,prefill,pack")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     args = ap.parse_args()

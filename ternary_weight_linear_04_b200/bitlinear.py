@@ -96,7 +96,8 @@ def forward(xq, eta, xsum, packed, gamma, N, out_dtype=torch.bfloat16, want_int=
 
 def fused_decode_ok(M, K):
     """Whether bitlinear_linear runs its single fused decode kernel for (M, K)
-    (the same rule as the library; otherwise it needs x~ scratch)."""
+    with bf16 activations (the same rule as the library; otherwise it needs
+    x~ scratch)."""
     mt = 1 if M <= 1 else (2 if M <= 2 else 4)
     return 1 <= M <= 4 and K % 64 == 0 and K * mt <= 32768
 
@@ -113,7 +114,7 @@ def linear(x, packed, gamma, N, out_dtype=torch.bfloat16, want_quant=False, want
         raise ValueError("packed shape %s does not match N=%d, K=%d" % (tuple(packed.shape), N, K))
     dev = x.device
     y = out if out is not None else torch.empty((M, N), dtype=out_dtype, device=dev)
-    decode = fused_decode_ok(M, K)
+    decode = fused_decode_ok(M, K) and x.dtype == torch.bfloat16
     if scratch is not None:
         xq, eta, xsum = scratch
     elif want_quant or not decode:

@@ -10,6 +10,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <type_traits>
 #include <utility>
 
 #include "bitlinear.h"
@@ -184,7 +185,9 @@ bl_status launch_decode_kernel(const bl::DecodeArgs& a0, int sms, cudaStream_t s
   if (stages > chunks) stages = chunks;
   if (stages < 1) stages = 1;
   a.stages = static_cast<int>(stages);
+  constexpr int64_t kXElem = std::is_same<XT, bl::DecNoFuse>::value ? 1 : 2;
   const size_t smem = static_cast<size_t>(nwj * MT * bl::kDecColThreads * 16) +
+                      static_cast<size_t>((MT * a.K * kXElem + 127) & ~int64_t{127}) +
                       static_cast<size_t>(stages * rps * P) + sizeof(bl::DecTail);
   auto kern = bl::k_decode<MT, XT, OutT>;
   if (!ensure_smem(kern, 227 * 1024, smem_done)) return BL_ERR_CUDA;
@@ -224,8 +227,9 @@ bl_status launch_generic(const int8_t* xq, const float* eta, int64_t M, int64_t 
 }
 
 template <int BM, typename OutT>
-bl_status launch_tc_bm(const int8_t* xq, const float* eta, int M, int K, const uint8_t* packed,
-                       const float* gamma, int N, void* y, int32_t* y_int, cudaStream_t st) {
+bl_status launch_tc_bm(const int8_t* xq, const float* eta, const int32_t* xsum, int M, int K,
+                       const uint8_t* packed, const float* gamma, int N, void* y, int32_t* y_int,
+                       cudaStream_t st) {
   using Cfg = bl::TcCfg<BM>;
   static int smem_done[kMaxDevices] = {0};
   auto kern = bl::k_gemm_tc<BM, OutT>;
@@ -238,17 +242,19 @@ bl_status launch_tc_bm(const int8_t* xq, const float* eta, int M, int K, const u
     return BL_ERR_CUDA;
   dim3 grid((N + bl::kTcBN - 1) / bl::kTcBN, (M + BM - 1) / BM);
   if (grid.y > 65535) return BL_ERR_UNSUPPORTED;
-  return launch_pdl(kern, grid, dim3(192), Cfg::kSmem, st, tm_x, tm_w, eta, gamma, M, K, N, y, y_int);
+  return launch_pdl(kern, grid, dim3(bl::kTcThreads), Cfg::kSmem, st, tm_x, tm_w, eta, xsum, gamma,
+                    M, K, N, y, y_int);
 }
 
 template <typename OutT>
-bl_status launch_tc(const int8_t* xq, const float* eta, int M, int K, const uint8_t* packed,
-                    const float* gamma, int N, void* y, int32_t* y_int, cudaStream_t st) {
-  if (M <= 16) return launch_tc_bm<16, OutT>(xq, eta, M, K, packed, gamma, N, y, y_int, st);
-  if (M <= 32) return launch_tc_bm<32, OutT>(xq, eta, M, K, packed, gamma, N, y, y_int, st);
-  if (M <= 64) return launch_tc_bm<64, OutT>(xq, eta, M, K, packed, gamma, N, y, y_int, st);
-  if (M <= 128) return launch_tc_bm<128, OutT>(xq, eta, M, K, packed, gamma, N, y, y_int, st);
-  return launch_tc_bm<256, OutT>(xq, eta, M, K, packed, gamma, N, y, y_int, st);
+bl_status launch_tc(const int8_t* xq, const float* eta, const int32_t* xsum, int M, int K,
+                    const uint8_t* packed, const float* gamma, int N, void* y, int32_t* y_int,
+                    cudaStream_t st) {
+  if (M <= 16) return launch_tc_bm<16, OutT>(xq, eta, xsum, M, K, packed, gamma, N, y, y_int, st);
+  if (M <= 32) return launch_tc_bm<32, OutT>(xq, eta, xsum, M, K, packed, gamma, N, y, y_int, st);
+  if (M <= 64) return launch_tc_bm<64, OutT>(xq, eta, xsum, M, K, packed, gamma, N, y, y_int, st);
+  if (M <= 128) return launch_tc_bm<128, OutT>(xq, eta, xsum, M, K, packed, gamma, N, y, y_int, st);
+  return launch_tc_bm<256, OutT>(xq, eta, xsum, M, K, packed, gamma, N, y, y_int, st);
 }
 
 bool fast_layout_ok(int64_t K, const void* xq, const void* packed, const void* y, const void* y_int) {
@@ -297,8 +303,9 @@ bl_status forward_impl(const int8_t* xq, const float* eta, const int32_t* xsum, 
         K > (1 << 30))
       return BL_ERR_UNSUPPORTED;
     return ydt == BL_F32
-               ? launch_tc<float>(xq, eta, (int)M, (int)K, packed, gamma, (int)N, y, y_int, s)
-               : launch_tc<__nv_bfloat16>(xq, eta, (int)M, (int)K, packed, gamma, (int)N, y, y_int, s);
+               ? launch_tc<float>(xq, eta, xsum, (int)M, (int)K, packed, gamma, (int)N, y, y_int, s)
+               : launch_tc<__nv_bfloat16>(xq, eta, xsum, (int)M, (int)K, packed, gamma, (int)N, y,
+                                          y_int, s);
   }
   return ydt == BL_F32
              ? launch_generic<float>(xq, eta, M, K, packed, gamma, N, y, y_int, sms, s)
@@ -479,7 +486,7 @@ bl_status bitlinear_linear(const void* x, bl_dtype xdt, int64_t M, int64_t K, co
   if (M == 0) return BL_OK;
   if (!x || !y) return BL_ERR_INVALID_ARG;
   if (127 * K >= (int64_t{1} << 31)) return BL_ERR_UNSUPPORTED;
-  const bool fused = decode_ok(M, K) &&
+  const bool fused = decode_ok(M, K) && xdt == BL_BF16 &&
                      aligned(x, 16) && aligned(packed, 16) && aligned(y, 16) &&
                      (!y_int || aligned(y_int, 16)) && (!xq || aligned(xq, 16)) &&
                      (!eta || aligned(eta, 4)) && (!xsum || aligned(xsum, 4)) && N <= INT32_MAX / 2;
@@ -500,11 +507,8 @@ bl_status bitlinear_linear(const void* x, bl_dtype xdt, int64_t M, int64_t K, co
   a.weights_static = (flags & BL_FLAG_WEIGHTS_STATIC) ? 1 : 0;
   a.xq_out = xq; a.eta_out = eta; a.xsum_out = xsum;
   const cudaStream_t s = as_stream(stream);
-  if (xdt == BL_BF16)
-    return ydt == BL_F32 ? launch_decode<__nv_bfloat16, float>(a, sms, s)
-                         : launch_decode<__nv_bfloat16, __nv_bfloat16>(a, sms, s);
-  return ydt == BL_F32 ? launch_decode<float, float>(a, sms, s)
-                       : launch_decode<float, __nv_bfloat16>(a, sms, s);
+  return ydt == BL_F32 ? launch_decode<__nv_bfloat16, float>(a, sms, s)
+                       : launch_decode<__nv_bfloat16, __nv_bfloat16>(a, sms, s);
 }
 
 bl_path bitlinear_select_path(int64_t M, int64_t K, int64_t N, const void* xq, const void* packed,

@@ -217,6 +217,11 @@ __host__ __device__ constexpr uint32_t make_idesc_i8(uint32_t M, uint32_t N) {
   return (2u << 4) | (1u << 7) | (1u << 10) | ((N >> 3) << 17) | ((M >> 4) << 24);
 }
 
+// The same with A unsigned 8-bit (a_format 0) and B signed 8-bit.
+__host__ __device__ constexpr uint32_t make_idesc_i8_u8s8(uint32_t M, uint32_t N) {
+  return (2u << 4) | (0u << 7) | (1u << 10) | ((N >> 3) << 17) | ((M >> 4) << 24);
+}
+
 // ---------------------------------------------------------------- misc
 
 __device__ __forceinline__ uint4 ld_nc_na_v4(const void* p) {

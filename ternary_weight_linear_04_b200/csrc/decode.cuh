@@ -79,34 +79,20 @@ __device__ __forceinline__ uint32_t pack4_i8(int32_t a, int32_t b, int32_t c, in
          ((static_cast<uint32_t>(c) & 0xFFu) << 16) | (static_cast<uint32_t>(d) << 24);
 }
 
-template <typename XT>
-struct DecLoad16;
-template <>
-struct DecLoad16<__nv_bfloat16> {
-  __device__ static void load(const void* p, float (&f)[16]) {
-    const uint4* q = static_cast<const uint4*>(p);
-    const uint4 a = __ldg(q), b = __ldg(q + 1);
-    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      f[2 * i] = __uint_as_float(w[i] << 16);
-      f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-    }
-  }
-};
-template <>
-struct DecLoad16<float> {
-  __device__ static void load(const void* p, float (&f)[16]) {
-    const float4* q = static_cast<const float4*>(p);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float4 v = __ldg(q + i);
-      f[4 * i] = v.x; f[4 * i + 1] = v.y; f[4 * i + 2] = v.z; f[4 * i + 3] = v.w;
-    }
-  }
-};
 // x~ given (not fused): the int8 activations themselves.
 struct DecNoFuse {};
+
+// 16 bf16 values from shared memory, widened to fp32 exactly.
+__device__ __forceinline__ void load16_bf16_smem(const uint8_t* p, float (&f)[16]) {
+  const uint4 a = *reinterpret_cast<const uint4*>(p);
+  const uint4 b = *reinterpret_cast<const uint4*>(p + 16);
+  const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
 
 struct DecodeArgs {
   const void* x;         // activations (fused) or x~ (int8), M x K
@@ -133,8 +119,10 @@ constexpr int kDecMaxChunks = 64;  // row chunks per CTA (the host sizes the gri
 struct DecTail {
   uint64_t full[kDecMaxStages];
   uint64_t empty[kDecMaxStages];
+  uint64_t xfull;  // the activation rows are in xbuf
   int abort_flag;
-  int pad[3];
+  float gamma;
+  int pad[2];
   float s_max[kDecComputeWarps][8];
   float s_scale[8];
   int32_t s_xsum[8];
@@ -198,7 +186,11 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode(const DecodeArgs a) {
   const int S = a.stages;
   const int stage_bytes = a.rows_per_stage * P;
   uint4* xslot = reinterpret_cast<uint4*>(smem);  // [nwj][MT][256 columns]
-  uint8_t* stages = smem + nwj * MT * kDecColThreads * 16;
+  // the M activation rows as given (bf16, or int8 x~), copied in one bulk copy
+  constexpr int kXElem = kFused ? 2 : 1;
+  uint8_t* xbuf = smem + nwj * MT * kDecColThreads * 16;
+  const int xbytes = a.M * K * kXElem;
+  uint8_t* stages = xbuf + ((MT * K * kXElem + 127) & ~127);
   DecTail& T = *reinterpret_cast<DecTail*>(stages + S * stage_bytes);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -224,11 +216,15 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode(const DecodeArgs a) {
         mbar_init(&T.full[s], 1);
         mbar_init(&T.empty[s], kDecComputeWarps);
       }
+      mbar_init(&T.xfull, 1);
       T.abort_flag = 0;
       mbar_init_fence();
       if (a.weights_static)
         for (int c = 0; c < first; ++c) issue(c);
       pdl_wait();  // the preceding grid is complete and its writes are visible
+      mbar_arrive_expect_tx(&T.xfull, static_cast<uint32_t>(xbytes));
+      bulk_load_1d(xbuf, a.x, static_cast<uint32_t>(xbytes), &T.xfull);
+      T.gamma = *a.gamma;
       if (!a.weights_static)
         for (int c = 0; c < first; ++c) issue(c);
     }
@@ -252,9 +248,11 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode(const DecodeArgs a) {
   for (int i = tid; i < nchunks; i += kDecComputeThreads) T.cnt[i] = 0;
   if (tid < 8) T.s_xsum[tid] = 0;
   named_sync(3, kDecThreads);  // wait for the producer: inputs of earlier kernels are visible
-  const float gamma = *a.gamma;
+  const float gamma = T.gamma;
+  const bool x_ok =
+      __all_sync(0xFFFFFFFFu, mbar_wait(&T.xfull, 0, &T.abort_flag));  // activations in xbuf
   if constexpr (kFused) {
-    const XT* x = static_cast<const XT*>(a.x);
+    static_assert(sizeof(XT) == 2, "the fused decode quantiser takes bf16 activations");
     // Word slots j are split between the teams: team t takes j = t, t+2, ...
 #pragma unroll
     for (int m = 0; m < MT; ++m) {
@@ -264,7 +262,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode(const DecodeArgs a) {
         const int w = ct + j * kDecColThreads;
         if (m < a.M && w < NW) {
           float f[16];
-          DecLoad16<XT>::load(x + static_cast<int64_t>(m) * K + 16 * w, f);
+          load16_bf16_smem(xbuf + (m * K + 16 * w) * 2, f);
 #pragma unroll
           for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(f[i]));
         }
@@ -288,7 +286,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode(const DecodeArgs a) {
         uint32_t q0 = 0, q1 = 0, q2 = 0, q3 = 0;
         if (m < a.M && w < NW) {
           float f[16];
-          DecLoad16<XT>::load(x + static_cast<int64_t>(m) * K + 16 * w, f);  // L1 hit
+          load16_bf16_smem(xbuf + (m * K + 16 * w) * 2, f);
           int32_t q[16];
           quantise16(f, eta, rcp, q);
 #pragma unroll
@@ -314,15 +312,13 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode(const DecodeArgs a) {
       }
     }
   } else {
-    const int8_t* xq = static_cast<const int8_t*>(a.x);
 #pragma unroll 1
     for (int j = team; j < nwj; j += kDecTeams)
 #pragma unroll
       for (int m = 0; m < MT; ++m) {
         const int w = ct + j * kDecColThreads;
         uint4 v = make_uint4(0, 0, 0, 0);
-        if (m < a.M && w < NW)
-          v = __ldg(reinterpret_cast<const uint4*>(xq + static_cast<int64_t>(m) * K) + w);
+        if (m < a.M && w < NW) v = *reinterpret_cast<const uint4*>(xbuf + m * K + 16 * w);
         uint4 t;
         transpose4x4_bytes(v.x, v.y, v.z, v.w, t.x, t.y, t.z, t.w);
         xslot[(j * MT + m) * kDecColThreads + ct] = t;
@@ -334,7 +330,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode(const DecodeArgs a) {
   }
   named_sync(1, kDecComputeThreads);  // activation slots of both teams are complete
 
-  for (int c = 0; c < nchunks; ++c) {
+  for (int c = 0; c < (x_ok ? nchunks : 0); ++c) {
     const int s = c % S;
     const bool ok =
         __all_sync(0xFFFFFFFFu, mbar_wait(&T.full[s], static_cast<uint32_t>(c / S) & 1u, &T.abort_flag));
