@@ -192,7 +192,7 @@ bl_status bitlinear_forward(const int8_t* xq, const float* eta, const int32_t* x
  * bitlinear_forward with the accumulate kernel and flags chosen by the
  * caller.  BL_PATH_GEMV and BL_PATH_TCGEN05 return BL_ERR_UNSUPPORTED when
  * the inputs do not meet their layout needs (K % 64 == 0, 16-byte
- * alignment; for BL_PATH_GEMV also M <= 4 and K * M' <= 32768, M' = M
+ * alignment; for BL_PATH_GEMV also M <= 4 and K * M' <= 131072, M' = M
  * rounded up to 1, 2 or 4); the results of every path are identical.
  * flags: 0 or BL_FLAG_WEIGHTS_STATIC.
  */
@@ -214,7 +214,7 @@ bl_status bitlinear_forward_path(const int8_t* xq, const float* eta, const int32
  *   y, ydt, y_int     out  as for bitlinear_forward (y_int optional).
  *   xq, eta, xsum     out  the quantised activations (M x K int8, M fp32,
  *                          M int32).  For bf16 decode batches (M <= 4,
- *                          K % 64 == 0, K * M' <= 32768 with M' = M rounded
+ *                          K % 64 == 0, K * M' <= 131072 with M' = M rounded
  *                          up to 1, 2 or 4, 16-byte aligned x, packed, y) one
  *                          fused kernel runs and these are optional (NULL =
  *                          not written).  Otherwise two kernels run and they
@@ -226,6 +226,34 @@ bl_status bitlinear_linear(const void* x, bl_dtype xdt, int64_t M, int64_t K,
                            void* y, bl_dtype ydt,
                            int8_t* xq, float* eta, int32_t* xsum,
                            int32_t* y_int, unsigned flags, void* stream);
+
+/*
+ * Launch shape of the decode kernel (BL_PATH_GEMV and the fused decode of
+ * bitlinear_linear) for M tokens, K inputs and N outputs on the current
+ * device; fused = 1 for bitlinear_linear's fused kernel (bf16 activations),
+ * 0 for bitlinear_forward's.  The pages have no counterpart: this describes
+ * how the library spreads the add / subtract / skip accumulation over a
+ * GPU.  shape (host, 10 int32) receives: team_warps G (warps splitting one
+ * row block's K), rows_per_block RB, teams, words per lane, rows per CTA,
+ * CTAs, row blocks per ring stage, ring stages, activations staged in
+ * shared memory (0/1), shared memory bytes per CTA.
+ * Errors: BL_ERR_INVALID_ARG for shape == NULL or N < 1; BL_ERR_UNSUPPORTED
+ * when the decode kernel does not take (M, K) or the forced shape (below)
+ * does not fit; BL_ERR_CUDA / BL_ERR_UNSUPPORTED without a B200-class GPU.
+ */
+bl_status bitlinear_decode_shape(int64_t M, int64_t K, int64_t N, int fused, int32_t* shape);
+
+/*
+ * Force the decode kernel's shape for every later launch in this process:
+ * team_warps G in 1..16 and rows_per_block RB in {1, 2, 4, 8, 16} (RB * M'
+ * <= 16 with M' = M rounded up to 1, 2 or 4); 0 for either leaves that
+ * choice to the library (the default).  A forced shape that a launch cannot
+ * use makes that launch return BL_ERR_UNSUPPORTED.  Results are identical
+ * for every shape; this exists to test and tune the shapes.  Not
+ * synchronised with launches in flight on other host threads.
+ * Errors: BL_ERR_INVALID_ARG for values outside those ranges.
+ */
+bl_status bitlinear_set_decode_shape(int team_warps, int rows_per_block);
 
 /* The path bitlinear_forward would pick for these sizes and pointers. */
 bl_path bitlinear_select_path(int64_t M, int64_t K, int64_t N,

@@ -34,6 +34,8 @@ SIGNATURES = {
                               ctypes.c_uint, _P]),
     "bitlinear_select_path": (_I, [_I64, _I64, _I64, _P, _P, _P, _P]),
     "bitlinear_device_error": (_I, [_P, _P]),
+    "bitlinear_decode_shape": (_I, [_I64, _I64, _I64, _I, _P]),
+    "bitlinear_set_decode_shape": (_I, [_I, _I]),
 }
 
 _lib = None

@@ -99,7 +99,25 @@ def fused_decode_ok(M, K):
     with bf16 activations (the same rule as the library; otherwise it needs
     x~ scratch)."""
     mt = 1 if M <= 1 else (2 if M <= 2 else 4)
-    return 1 <= M <= 4 and K % 64 == 0 and K * mt <= 32768
+    return 1 <= M <= 4 and K >= 64 and K % 64 == 0 and K * mt <= 131072
+
+
+DECODE_SHAPE_FIELDS = ("team_warps", "rows_per_block", "teams", "words_per_lane", "rows_per_cta",
+                       "ctas", "blocks_per_stage", "stages", "x_staged", "smem_bytes")
+
+
+def decode_shape(M, K, N, fused=True):
+    """The decode kernel's launch shape for (M, K, N) on the current device,
+    as a dict (see bitlinear_decode_shape)."""
+    buf = (ctypes.c_int32 * len(DECODE_SHAPE_FIELDS))()
+    check(_lib.lib().bitlinear_decode_shape(M, K, N, 1 if fused else 0, buf), "bitlinear_decode_shape")
+    return dict(zip(DECODE_SHAPE_FIELDS, list(buf)))
+
+
+def set_decode_shape(team_warps=0, rows_per_block=0):
+    """Force the decode kernel's team width and row-block height for later
+    launches in this process (0 = the library's choice)."""
+    check(_lib.lib().bitlinear_set_decode_shape(team_warps, rows_per_block), "bitlinear_set_decode_shape")
 
 
 def linear(x, packed, gamma, N, out_dtype=torch.bfloat16, want_quant=False, want_int=False,

@@ -9,6 +9,7 @@
 
 #include <cstdint>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 #include <type_traits>
 #include <utility>
@@ -30,10 +31,10 @@ constexpr int kGemvMaxM = 4;  // largest token count the CUDA-core decode kernel
 inline int decode_mt(int64_t M) { return M <= 1 ? 1 : (M <= 2 ? 2 : 4); }
 
 // Whether the decode kernel takes (M, K): K % 64 == 0, M <= 4 and
-// K * MT <= 32768 (each thread stages at most 8 words x MT tokens of
-// activations, 32 KB of shared memory per CTA).
+// K * MT <= 131072 (the quantised activations of all MT tokens sit in
+// shared memory, K * MT bytes, beside at least one ring stage).
 inline bool decode_ok(int64_t M, int64_t K) {
-  return M >= 1 && M <= kGemvMaxM && K % 64 == 0 && K * decode_mt(M) <= 32768;
+  return M >= 1 && M <= kGemvMaxM && K >= 64 && K % 64 == 0 && K * decode_mt(M) <= 131072;
 }
 
 inline bool aligned(const void* p, uintptr_t a) {
@@ -156,42 +157,148 @@ bool make_tmap_u8(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t col
 // ------------------------------------------------------------ launchers
 
 // Decode kernel (M <= 4 tokens): one CTA per SM, each owning a contiguous
-// block of rows, so the next kernel's CTA fits beside it under programmatic
-// dependent launch.  XT = activation type when the quantiser is fused, or
-// bl::DecNoFuse when x~ is given.
-template <int MT, typename XT, typename OutT>
-bl_status launch_decode_kernel(const bl::DecodeArgs& a0, int sms, cudaStream_t st) {
-  static int smem_done[kMaxDevices] = {0};
-  bl::DecodeArgs a = a0;
-  const int64_t P = a.K / 4;
-  const int64_t nwj = (a.K / 16 + bl::kDecColThreads - 1) / bl::kDecColThreads;
-  int64_t rps = bl::kDecStageTarget / P;  // rows per stage (one chunk)
-  if (rps > 32 / MT) rps = 32 / MT;
-  if (rps < 1) rps = 1;
-  // One CTA per SM, unless that would give a CTA more chunks than its
-  // reduction slots hold.
-  int64_t grid = sms;
-  const int64_t min_grid = (a.N + rps * bl::kDecMaxChunks - 1) / (rps * bl::kDecMaxChunks);
-  if (grid < min_grid) grid = min_grid;
-  if (grid > a.N) grid = a.N;
-  a.rows_per_cta = static_cast<int>((a.N + grid - 1) / grid);
-  grid = (a.N + a.rows_per_cta - 1) / a.rows_per_cta;
-  if (rps > a.rows_per_cta) rps = a.rows_per_cta;
-  a.rows_per_stage = static_cast<int>(rps);
-  const int64_t chunks = (a.rows_per_cta + rps - 1) / rps;
-  if (chunks > bl::kDecMaxChunks || grid > 0x7FFFFFFF) return BL_ERR_UNSUPPORTED;
-  int64_t stages = bl::kDecSmemBudget / (rps * P);
+// range of rows, small enough that the next kernel's CTA fits beside it
+// under programmatic dependent launch.
+//
+// The shape of the work inside a CTA -- G warps per team splitting K, RB
+// rows per block -- is picked here by a small cost model in SM cycles: the
+// largest of (instructions / 4 issue slots, dp4a / 2 per cycle, shared
+// memory wavefronts, and 2 x one warp's own instruction stream), with the
+// padding words (32*G*nwj >= K/16) and padding rows (blocks of RB) counted.
+struct DecGeom {
+  int G = 1, teams = 16, nwj = 1, RB = 1;
+  int rows_per_cta = 1, grid = 1, bpc = 1, stages = 1, x_staged = 0;
+  size_t smem = 0;
+};
+
+constexpr size_t kDecTwoCtaSmem = 113 * 1024;  // two CTAs per SM (228 KB less 1 KB each)
+constexpr size_t kDecMaxSmem = 227 * 1024;
+constexpr int64_t kDecRingBytes = 64 * 1024;
+constexpr int64_t kDecStageTarget = 32 * 1024;
+
+inline bool rb_allowed(int MT, int RB) { return RB * MT <= 16; }
+
+// Shape forced by bitlinear_set_decode_shape (0 = chosen by the model).
+std::atomic<int> g_force_G{0}, g_force_RB{0};
+
+bool decode_geometry(int MT, int64_t M, int64_t K, int64_t N, int sms, int64_t xelem,
+                     DecGeom* out) {
+  const int64_t NW = K / 16, P = K / 4;
+  const int fG = g_force_G.load(std::memory_order_relaxed);
+  const int fRB = g_force_RB.load(std::memory_order_relaxed);
+  int64_t grid = N < sms ? N : sms;
+  int64_t rpc = (N + grid - 1) / grid;
+  grid = (N + rpc - 1) / rpc;
+  double best = 1e30;
+  bool found = false;
+  for (int RB = 1; RB <= 16; RB *= 2) {
+    if (!rb_allowed(MT, RB) || (fRB && RB != fRB)) continue;
+    const int V = RB * MT;
+    const int alu = V <= 8 ? 5 : 7;
+    const int64_t nblocks = (rpc + RB - 1) / RB;
+    for (int G = 1; G <= 16; ++G) {
+      if (fG && G != fG) continue;
+      const int teams = 16 / G;
+      if (G > 1 && nblocks > bl::kDecMaxBlocks) continue;
+      const int64_t nwj = (NW + 32 * G - 1) / (32 * G);
+      const int64_t bpt = (nblocks + teams - 1) / teams;
+      // per warp and block: x~ loads, weight loads, plane split, dp4a, loop
+      const double per_block = nwj * (MT + RB + alu * RB + 4.0 * V + 3) + 2.0 * V + 8 +
+                               (G > 1 ? 10 : 0);
+      const double warp_blocks = static_cast<double>(nblocks) * G;
+      const double t_issue = warp_blocks * per_block / 4.0;
+      const double t_dp4a = warp_blocks * nwj * 4.0 * V / 2.0;
+      const double t_lsu = warp_blocks * nwj * (4.0 * MT + RB);
+      const double t_warp = 2.0 * bpt * per_block;
+      double cost = t_issue;
+      if (t_dp4a > cost) cost = t_dp4a;
+      if (t_lsu > cost) cost = t_lsu;
+      if (t_warp > cost) cost = t_warp;
+      // shared memory: slots + ring of at least one block + tail
+      const int64_t slots = static_cast<int64_t>(MT) * 32 * G * nwj * 16;
+      const int64_t blk = RB * P;
+      if (slots + blk + static_cast<int64_t>(sizeof(bl::DecTail)) > static_cast<int64_t>(kDecMaxSmem))
+        continue;
+      if (cost < best * 0.999) {
+        best = cost;
+        found = true;
+        out->G = G; out->teams = teams; out->nwj = static_cast<int>(nwj); out->RB = RB;
+      }
+    }
+  }
+  if (!found) return false;
+  // ring: whole blocks per stage, about kDecStageTarget per stage
+  const int64_t blk = out->RB * P;
+  const int64_t nblocks = (rpc + out->RB - 1) / out->RB;
+  int64_t bpc = kDecStageTarget / blk;
+  if (bpc < 1) bpc = 1;
+  if (bpc > nblocks) bpc = nblocks;
+  const int64_t chunks = (nblocks + bpc - 1) / bpc;
+  const int64_t slots = static_cast<int64_t>(MT) * 32 * out->G * out->nwj * 16;
+  const int64_t tail = static_cast<int64_t>(sizeof(bl::DecTail));
+  const int64_t xbytes = ((M * K * xelem) + 127) & ~int64_t{127};
+  int64_t ring = kDecRingBytes;
+  // stay within two CTAs per SM when the slots allow it
+  if (slots + tail + bpc * blk <= static_cast<int64_t>(kDecTwoCtaSmem) &&
+      slots + tail + ring > static_cast<int64_t>(kDecTwoCtaSmem))
+    ring = static_cast<int64_t>(kDecTwoCtaSmem) - slots - tail;
+  if (slots + tail + ring > static_cast<int64_t>(kDecMaxSmem))
+    ring = static_cast<int64_t>(kDecMaxSmem) - slots - tail;
+  int64_t stages = ring / (bpc * blk);
   if (stages > bl::kDecMaxStages) stages = bl::kDecMaxStages;
   if (stages > chunks) stages = chunks;
   if (stages < 1) stages = 1;
-  a.stages = static_cast<int>(stages);
+  size_t smem = static_cast<size_t>(slots + stages * bpc * blk + tail);
+  int x_staged = 0;
+  const size_t limit = smem <= kDecTwoCtaSmem ? kDecTwoCtaSmem : kDecMaxSmem;
+  if (smem + static_cast<size_t>(xbytes) <= limit) {
+    smem += static_cast<size_t>(xbytes);
+    x_staged = 1;
+  }
+  if (smem > kDecMaxSmem) return false;
+  out->rows_per_cta = static_cast<int>(rpc);
+  out->grid = static_cast<int>(grid);
+  out->bpc = static_cast<int>(bpc);
+  out->stages = static_cast<int>(stages);
+  out->x_staged = x_staged;
+  out->smem = smem;
+  return true;
+}
+
+template <int MT, int RB, typename XT, typename OutT>
+bl_status launch_decode_rb(const bl::DecodeArgs& a, const DecGeom& g, cudaStream_t st) {
+  static int smem_done[kMaxDevices] = {0};
+  auto kern = bl::k_decode<MT, RB, XT, OutT>;
+  if (!ensure_smem(kern, static_cast<int>(kDecMaxSmem), smem_done)) return BL_ERR_CUDA;
+  return launch_pdl(kern, dim3(static_cast<unsigned>(g.grid)), dim3(bl::kDecThreads), g.smem, st,
+                    a);
+}
+
+template <int MT, typename XT, typename OutT>
+bl_status launch_decode_kernel(const bl::DecodeArgs& a0, int sms, cudaStream_t st) {
   constexpr int64_t kXElem = std::is_same<XT, bl::DecNoFuse>::value ? 1 : 2;
-  const size_t smem = static_cast<size_t>(nwj * MT * bl::kDecColThreads * 16) +
-                      static_cast<size_t>((MT * a.K * kXElem + 127) & ~int64_t{127}) +
-                      static_cast<size_t>(stages * rps * P) + sizeof(bl::DecTail);
-  auto kern = bl::k_decode<MT, XT, OutT>;
-  if (!ensure_smem(kern, 227 * 1024, smem_done)) return BL_ERR_CUDA;
-  return launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(bl::kDecThreads), smem, st, a);
+  DecGeom g;
+  if (!decode_geometry(MT, a0.M, a0.K, a0.N, sms, kXElem, &g)) return BL_ERR_UNSUPPORTED;
+  bl::DecodeArgs a = a0;
+  a.rows_per_cta = g.rows_per_cta;
+  a.blocks_per_chunk = g.bpc;
+  a.stages = g.stages;
+  a.team_warps = g.G;
+  a.teams = g.teams;
+  a.nwj = g.nwj;
+  a.x_staged = g.x_staged;
+  switch (g.RB) {
+    case 1: return launch_decode_rb<MT, 1, XT, OutT>(a, g, st);
+    case 2: return launch_decode_rb<MT, 2, XT, OutT>(a, g, st);
+    case 4: return launch_decode_rb<MT, 4, XT, OutT>(a, g, st);
+    case 8:
+      if constexpr (MT <= 2) return launch_decode_rb<MT, 8, XT, OutT>(a, g, st);
+      break;
+    case 16:
+      if constexpr (MT == 1) return launch_decode_rb<MT, 16, XT, OutT>(a, g, st);
+      break;
+  }
+  return BL_ERR_UNSUPPORTED;
 }
 
 template <typename XT, typename OutT>
@@ -326,6 +433,36 @@ const char* bitlinear_status_str(bl_status status) {
     case BL_ERR_TIMEOUT: return "a kernel gave up a bounded wait";
   }
   return "unknown status";
+}
+
+bl_status bitlinear_decode_shape(int64_t M, int64_t K, int64_t N, int fused, int32_t* shape) {
+  if (!shape || N < 1) return BL_ERR_INVALID_ARG;
+  if (!decode_ok(M, K) || N > INT32_MAX / 2) return BL_ERR_UNSUPPORTED;
+  int sms = 148;
+  const bl_status st = device_info(&sms);
+  if (st != BL_OK) return st;
+  DecGeom g;
+  if (!decode_geometry(decode_mt(M), M, K, N, sms, fused ? 2 : 1, &g)) return BL_ERR_UNSUPPORTED;
+  shape[0] = g.G;
+  shape[1] = g.RB;
+  shape[2] = g.teams;
+  shape[3] = g.nwj;
+  shape[4] = g.rows_per_cta;
+  shape[5] = g.grid;
+  shape[6] = g.bpc;
+  shape[7] = g.stages;
+  shape[8] = g.x_staged;
+  shape[9] = static_cast<int32_t>(g.smem);
+  return BL_OK;
+}
+
+bl_status bitlinear_set_decode_shape(int team_warps, int rows_per_block) {
+  if (team_warps < 0 || team_warps > 16) return BL_ERR_INVALID_ARG;
+  if (rows_per_block < 0 || rows_per_block > 16 || (rows_per_block & (rows_per_block - 1)) != 0)
+    return BL_ERR_INVALID_ARG;
+  g_force_G.store(team_warps, std::memory_order_relaxed);
+  g_force_RB.store(rows_per_block, std::memory_order_relaxed);
+  return BL_OK;
 }
 
 const char* bitlinear_version(void) { return "0.1.0"; }

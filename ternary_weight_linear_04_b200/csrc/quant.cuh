@@ -10,6 +10,8 @@
 // (sum x~ * t = sum x~ * c - sum x~).
 #pragma once
 
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace bl {
@@ -26,48 +28,95 @@ __device__ __forceinline__ float load_as_f32<__nv_bfloat16>(const __nv_bfloat16*
 // x~ = clip(RNE(RN32(RN32(x * 127) / eta)), -127, 127), computed exactly but
 // without a division per element.  Only the integer RNE(q) is needed, and it
 // only depends on which side of the nearest half-integer q falls.  With
-// rcp = RN32(1/eta) the product q' = RN32(a * rcp) is within 2^-23 * |a/eta|
-// <= 1.6e-5 of a/eta, and q = RN32(a/eta) within 3.9e-6 of it (|a/eta| <=
-// 127), so |q - q'| < 2e-5.  If q' is farther than 2^-14 (6.1e-5) from its
-// nearest half-integer, q lies strictly on the same side and RNE(q) =
-// RNE(q'); otherwise the IEEE quotient itself is formed.
+// s = RN32(127 * RN32(1/eta)), the product c = RN32(x * s) differs from
+// 127x/eta by a relative error of at most 3 roundings, and q = RN32(a/eta)
+// (a = RN32(127x)) by at most 2, so |c - q| <= 127 * 5 * 2^-24 < 3.8e-5
+// (|x| <= eta).  If c is farther than 2^-14 (6.1e-5) from its nearest
+// half-integer, q lies strictly on the same side and RNE(q) = RNE(c);
+// otherwise the IEEE quotient itself is formed.  |c| < 127.5, so the clip
+// never binds on the fast path.
+//
+// RNE(c) comes from the fp32 adder, not the conversion unit: for |c| < 2^22,
+// t = RN32(c + 1.5 * 2^23) lies on the integer grid of [2^23, 2^24), so t's
+// low mantissa bits hold RNE(c) in two's complement (its low byte is the
+// int8 code) and t - 1.5 * 2^23 is RNE(c) exactly; c - RNE(c) is exact too
+// (the operands are within a factor of two, or RNE(c) = 0).
+constexpr float kRneMagic = 12582912.0f;        // 1.5 * 2^23
+constexpr uint32_t kRneMagicBits = 0x4B400000u;  // its bit pattern
+constexpr float kTieGuard = 0.49993896484375f;   // 0.5 - 2^-14
+
 // The exact quotient, out of line so the common path stays a few instructions
 // and the divide is a real (rarely taken) branch rather than predicated code.
 __device__ __noinline__ float quotient_exact(float a, float eta) { return __fdiv_rn(a, eta); }
 
-__device__ __forceinline__ int32_t quantise_fast(float x, float eta, float rcp) {
-  const float a = __fmul_rn(x, 127.0f);
-  float q = __fmul_rn(a, rcp);
-  const float fr = q - floorf(q);
-  if (fabsf(fr - 0.5f) < 6.103515625e-05f) q = quotient_exact(a, eta);
-  const float r = fminf(fmaxf(rintf(q), -127.0f), 127.0f);  // rintf: nearest, ties to even
-  return static_cast<int32_t>(r);
+// Scale for the fast path: RN32(127 * RN32(1 / eta)).
+__device__ __forceinline__ float quant_scale(float eta) {
+  return __fmul_rn(127.0f, __frcp_rn(eta));
 }
 
-// The same for 16 values at once, with no branch in the common path: all 16
-// candidates are formed first, and only if some lane of the warp has a value
-// near a tie does the warp take the (rare) exact fix-up loop.
-__device__ __forceinline__ void quantise16(const float (&f)[16], float eta, float rcp,
-                                           int32_t (&q)[16]) {
-  float a[16];
-  uint32_t near = 0;
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    a[i] = __fmul_rn(f[i], 127.0f);
-    const float c = __fmul_rn(a[i], rcp);
-    const float fr = c - floorf(c);
-    near |= (fabsf(fr - 0.5f) < 6.103515625e-05f ? 1u : 0u) << i;
-    q[i] = static_cast<int32_t>(fminf(fmaxf(rintf(c), -127.0f), 127.0f));
-  }
-  if (__any_sync(__activemask(), near != 0)) {
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      if ((near >> i) & 1u) {
-        const float c = quotient_exact(a[i], eta);
-        q[i] = static_cast<int32_t>(fminf(fmaxf(rintf(c), -127.0f), 127.0f));
-      }
-    }
-  }
+// The exact code of one value, as the bit pattern of RNE(q) + 1.5 * 2^23.
+__device__ __forceinline__ uint32_t quantise_exact_bits(float x, float eta) {
+  const float q = quotient_exact(__fmul_rn(x, 127.0f), eta);
+  return __float_as_uint(__fadd_rn(fminf(fmaxf(rintf(q), -127.0f), 127.0f), kRneMagic));
+}
+
+__device__ __forceinline__ int32_t quantise_fast(float x, float eta, float s) {
+  const float c = __fmul_rn(x, s);
+  float t = __fadd_rn(c, kRneMagic);
+  const float d = __fsub_rn(c, __fsub_rn(t, kRneMagic));
+  uint32_t bits = __float_as_uint(t);
+  if (fabsf(d) > kTieGuard) bits = quantise_exact_bits(x, eta);
+  return static_cast<int32_t>(bits - kRneMagicBits);
+}
+
+// bf16 activations, exactly, with no division and no branch.  When x and
+// eta are both bf16 values (eta >= 1e-5 is then one of the |x|):
+//   * a = 127x is exact in fp32 (8 x 7 significant bits);
+//   * for every half-integer h, a/eta is either exactly h or farther from h
+//     than 1/(2 * 255 * 2^9), far more than half an fp32 ulp of h (below
+//     2^-18): with x = mx 2^ex, eta = me 2^ee (8-bit integers mx, me),
+//     a/eta - h is an integer over 2 me 2^max(0, ee-ex), and exponent gaps of
+//     10 or more leave |a/eta| < 0.25, away from every h.  So RN32 keeps
+//     a/eta on its side of every h, and RNE(RN32(a/eta)) = RNE(a/eta) with
+//     ties (a/eta = h exactly) to even;
+//   * the fast candidate n0 = RNE(RN32(x * s)) is within 0.5 + 3.8e-5 of
+//     a/eta (see above), and e = a - n0 * eta is exact in fp32: n0 * eta has
+//     at most 15 significant bits, and the difference spans at most 24 bits
+//     (for x far below eta, n0 is 0 or +-1).  One fma forms it.
+// So RNE(a/eta) = n0 + 1 if e > eta/2, n0 - 1 if e < -eta/2, and on
+// |e| = eta/2 exactly (a tie) the even one of n0 and n0 + sign(e).  The
+// result is returned as the bit pattern of RNE + 1.5 * 2^23 (low byte = the
+// int8 code); |a/eta| <= 127, so it stays within [-127, 127].
+// heta = 0.5 * eta (exact).
+__device__ __forceinline__ uint32_t code_bits_bf16(float x, float eta, float heta, float s) {
+  const float t = __fadd_rn(__fmul_rn(x, s), kRneMagic);
+  const float n0 = __fsub_rn(t, kRneMagic);
+  const float e = __fmaf_rn(x, 127.0f, -__fmul_rn(n0, eta));
+  uint32_t bits = __float_as_uint(t);
+  bits += (e > heta) ? 1u : 0u;
+  bits -= (e < -heta) ? 1u : 0u;
+  if (fabsf(e) == heta && (bits & 1u)) bits += (e > 0.0f) ? 1u : 0xFFFFFFFFu;
+  return bits;
+}
+
+// Whether v is a bf16 value (its low 16 bits are zero).
+__device__ __forceinline__ bool is_bf16_value(float v) {
+  return (__float_as_uint(v) & 0xFFFFu) == 0;
+}
+
+// One bf16 activation (widened exactly to fp32).  When eta is the 1e-5
+// floor rather than a bf16 value (every |x| of the row below 1e-5), the
+// argument above does not hold and the code takes the IEEE quotient
+// (a uniform branch: eta is shared by the row).
+__device__ __forceinline__ int32_t quantise_bf16(float x, float eta, float s, bool eta_bf16) {
+  const uint32_t bits = eta_bf16 ? code_bits_bf16(x, eta, __fmul_rn(0.5f, eta), s)
+                                 : quantise_exact_bits(x, eta);
+  return static_cast<int32_t>(bits - kRneMagicBits);
+}
+
+// Low bytes of four words, in order, packed into one word.
+__device__ __forceinline__ uint32_t pack_lowbytes(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
 }
 
 // Block-wide reductions over 256 threads.
@@ -143,6 +192,7 @@ __global__ void __launch_bounds__(256) k_quant_act(const T* __restrict__ x, int6
   __shared__ float redf[8];
   __shared__ int32_t redi[8];
   constexpr int V = QVec<T>::kN;
+  constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   for (int64_t m = blockIdx.x; m < M; m += gridDim.x) {
@@ -161,7 +211,8 @@ __global__ void __launch_bounds__(256) k_quant_act(const T* __restrict__ x, int6
     }
     amax = block_max_256(amax, redf);
     const float eta = fmaxf(amax, 1e-5f);
-    const float rcp = __frcp_rn(eta);
+    const float qs = quant_scale(eta);
+    const bool eta_bf16 = is_bf16_value(eta);
     int32_t sum = 0;
     if (vec) {
       for (int64_t k = static_cast<int64_t>(threadIdx.x) * V; k < K; k += 256 * V) {
@@ -170,14 +221,15 @@ __global__ void __launch_bounds__(256) k_quant_act(const T* __restrict__ x, int6
         int32_t q[V];
 #pragma unroll
         for (int i = 0; i < V; ++i) {
-          q[i] = quantise_fast(f[i], eta, rcp);
+          q[i] = kBf16 ? quantise_bf16(f[i], eta, qs, eta_bf16) : quantise_fast(f[i], eta, qs);
           sum += q[i];
         }
         QVec<T>::store(qrow + k, q);
       }
     } else {
       for (int64_t k = threadIdx.x; k < K; k += 256) {
-        const int32_t q = quantise_fast(load_as_f32(row + k), eta, rcp);
+        const float xv = load_as_f32(row + k);
+        const int32_t q = kBf16 ? quantise_bf16(xv, eta, qs, eta_bf16) : quantise_fast(xv, eta, qs);
         sum += q;
         qrow[k] = static_cast<int8_t>(q);
       }

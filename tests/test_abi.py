@@ -80,6 +80,17 @@ def test_bad_arguments_are_rejected_without_a_launch(L):
     # a prefill-sized batch needs the caller's x~ scratch
     assert lin(fake, 1, 64, 64, fake, fake, 8, fake, 1, None, None, None, None, 0, None) == _lib.BL_ERR_INVALID_ARG
     assert L.bitlinear_device_error(None, None) == _lib.BL_ERR_INVALID_ARG
+    shape = (ctypes.c_int32 * 10)()
+    assert L.bitlinear_decode_shape(1, 3200, 8640, 1, None) == _lib.BL_ERR_INVALID_ARG
+    assert L.bitlinear_decode_shape(1, 3200, 0, 1, shape) == _lib.BL_ERR_INVALID_ARG
+    assert L.bitlinear_decode_shape(5, 3200, 8640, 1, shape) == _lib.BL_ERR_UNSUPPORTED   # M > 4
+    assert L.bitlinear_decode_shape(1, 3232, 8640, 1, shape) == _lib.BL_ERR_UNSUPPORTED   # K % 64
+    assert L.bitlinear_decode_shape(4, 65536, 64, 1, shape) == _lib.BL_ERR_UNSUPPORTED    # K * M'
+    assert L.bitlinear_set_decode_shape(17, 0) == _lib.BL_ERR_INVALID_ARG
+    assert L.bitlinear_set_decode_shape(-1, 0) == _lib.BL_ERR_INVALID_ARG
+    assert L.bitlinear_set_decode_shape(0, 3) == _lib.BL_ERR_INVALID_ARG
+    assert L.bitlinear_set_decode_shape(0, 32) == _lib.BL_ERR_INVALID_ARG
+    assert L.bitlinear_set_decode_shape(0, 0) == _lib.BL_OK
 
 
 def test_path_selection_is_host_logic(L):
@@ -87,6 +98,8 @@ def test_path_selection_is_host_logic(L):
     a = P(1 << 20)
     sel = L.bitlinear_select_path
     assert sel(1, 4096, 4096, a, a, a, None) == _lib.BL_PATH_GEMV
+    assert sel(1, 28672, 8192, a, a, a, None) == _lib.BL_PATH_GEMV      # K * M' <= 131072
+    assert sel(4, 65536, 64, a, a, a, None) == _lib.BL_PATH_TCGEN05     # K * M' > 131072
     assert sel(2048, 4096, 11008, a, a, a, None) == _lib.BL_PATH_TCGEN05
     assert sel(1, 4095, 4096, a, a, a, None) == _lib.BL_PATH_GENERIC      # ragged K
     assert sel(1, 4096, 4096, P((1 << 20) + 8), a, a, None) == _lib.BL_PATH_GENERIC  # misaligned

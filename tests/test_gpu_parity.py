@@ -333,11 +333,153 @@ def test_bitlinear_module():
 
 
 @pytest.mark.parametrize("M", [1, 2, 3, 4])
-@pytest.mark.parametrize("K", [64, 4096, 4160, 8192, 12288, 16384, 32768])
+@pytest.mark.parametrize("K", [64, 4096, 4160, 8192, 12288, 16384, 32768, 65536, 131072])
 def test_decode_word_widths(M, K):
-    """Every words-per-thread width (1, 2, 4, 8) and stage/row-block shape of
-    the decode kernel, with N not a multiple of the rows per CTA."""
-    if K * (1 if M == 1 else (2 if M == 2 else 4)) > 32768:
-        pytest.skip("outside the decode kernel's register budget")
+    """The decode kernel's own shape choice across K (padding words, ring
+    stages, activations staged in shared memory or read from global), with
+    N not a multiple of the rows per CTA."""
+    if K * (1 if M == 1 else (2 if M == 2 else 4)) > 131072:
+        pytest.skip("outside the decode kernel's shared-memory budget")
     W, x = inputs.make_case(9000 + M + K, M, K, 1237, act_dtype="bf16")
     check_layer(W, x, "bf16", "bf16", path="gemv")
+
+
+@pytest.fixture
+def forced_shape():
+    yield bl.set_decode_shape
+    bl.set_decode_shape(0, 0)
+
+
+def _shape_or_skip(M, K, N, fused):
+    try:
+        return bl.decode_shape(M, K, N, fused=fused)
+    except Exception as e:  # the forced shape cannot take this size
+        if getattr(e, "status", None) == 2:
+            pytest.skip("forced shape does not fit (M, K, N)")
+        raise
+
+
+@pytest.mark.parametrize("M", [1, 2, 3])
+@pytest.mark.parametrize("RB", [1, 2, 4, 8, 16])
+@pytest.mark.parametrize("G", [1, 2, 7, 16])
+@pytest.mark.parametrize("K,N", [(3200, 2000), (3200, 12400), (1024, 140)])
+def test_decode_forced_shapes(forced_shape, M, RB, G, K, N):
+    """Every (team width G, row block RB) instantiation of the decode kernel,
+    fused and not: padding words (K/16 = 200 words against 32*G*nwj slots),
+    partial row blocks, one row per CTA (N = 140), and a ring that wraps
+    (N = 12400: 84 rows of 800 bytes per CTA)."""
+    mt = 1 if M == 1 else (2 if M == 2 else 4)
+    if RB * mt > 16:
+        pytest.skip("RB * M' > 16")
+    forced_shape(G, RB)
+    shp = _shape_or_skip(M, K, N, True)
+    assert (shp["team_warps"], shp["rows_per_block"]) == (G, RB)
+    W, x = inputs.make_case(7000 + 17 * M + RB + 3 * G + N, M, K, N, act_dtype="bf16")
+    ref_packed, ref_gamma, _ = orc.pack_weights(W)
+    _, _, packed, gamma = gpu_pack(W)
+    ref_xq, ref_eta, ref_xsum = orc.quant_act(x)
+    ref_yint, ref_y = orc.forward(ref_xq, ref_eta, ref_packed, ref_gamma, K, N)
+    xd = torch.from_numpy(x).cuda().to(torch.bfloat16)
+    y, (xq, eta, xsum), y_int = bl.linear(xd, packed, gamma, N, out_dtype=torch.bfloat16,
+                                          want_quant=True, want_int=True, weights_static=True)
+    np.testing.assert_array_equal(xq.cpu().numpy(), ref_xq)
+    np.testing.assert_array_equal(xsum.cpu().numpy(), ref_xsum)
+    np.testing.assert_array_equal(y_int.cpu().numpy(), ref_yint)
+    np.testing.assert_array_equal(y_bits(y.cpu()), orc.f32_to_bf16_bits(ref_y))
+    _shape_or_skip(M, K, N, False)
+    xq_d = torch.from_numpy(ref_xq).cuda()
+    y2, y2_int = bl.forward(xq_d, torch.from_numpy(ref_eta).cuda(), torch.from_numpy(ref_xsum).cuda(),
+                            packed, gamma, N, out_dtype=torch.float32, want_int=True, path="gemv")
+    np.testing.assert_array_equal(y2_int.cpu().numpy(), ref_yint)
+    np.testing.assert_array_equal(y2.cpu().numpy().view(np.uint32), ref_y.view(np.uint32))
+
+
+def test_decode_shape_query_and_override(forced_shape):
+    shp = bl.decode_shape(1, 3200, 8640)
+    assert shp["team_warps"] * shp["teams"] <= 16 and shp["rows_per_block"] in (1, 2, 4, 8, 16)
+    assert shp["words_per_lane"] * 32 * shp["team_warps"] >= 3200 // 16
+    assert shp["rows_per_cta"] * shp["ctas"] >= 8640
+    forced_shape(3, 4)
+    shp = bl.decode_shape(1, 3200, 8640)
+    assert (shp["team_warps"], shp["rows_per_block"], shp["teams"]) == (3, 4, 5)
+    with pytest.raises(Exception):
+        forced_shape(17, 0)
+    with pytest.raises(Exception):
+        forced_shape(0, 3)
+
+
+# ----------------------------------------------------------------- exact ties of bf16 activations
+
+def _all_bf16_below(eta):
+    """Every bf16 value x with 0 < |x| < eta, both signs, then eta itself
+    first (so eta is the row's absmax)."""
+    bits = np.arange(1, 0x7F80, dtype=np.uint32)  # positive finite bf16 patterns
+    vals = (bits << 16).view(np.float32)
+    vals = vals[vals < eta]
+    return np.concatenate([[eta], vals, -vals]).astype(np.float32)
+
+
+def _tie_rows(mantissas, K):
+    rows = []
+    for m in mantissas:
+        eta = np.float32(m / 128.0)  # a bf16 value in [1, 2)
+        r = _all_bf16_below(eta)
+        assert r.size <= K
+        rows.append(np.concatenate([r, np.zeros(K - r.size, np.float32)]))
+    return np.stack(rows)
+
+
+def test_quantiser_exact_on_every_bf16_tie():
+    """For each of the 128 bf16 mantissas of eta in [1, 2), a row holding
+    every bf16 value below eta: 127x/eta hits every exact .5 tie and every
+    near tie the lattice of bf16 ratios can produce.  Standalone quantiser
+    (bf16 input) against the oracle's division."""
+    K = 34816
+    x = _tie_rows(range(128, 256), K)
+    ref_xq, ref_eta, ref_xsum = orc.quant_act(x)
+    xq, eta, xsum = gpu_quant(x, "bf16")
+    np.testing.assert_array_equal(eta.cpu().numpy(), ref_eta)
+    np.testing.assert_array_equal(xq.cpu().numpy(), ref_xq)
+    np.testing.assert_array_equal(xsum.cpu().numpy(), ref_xsum)
+
+
+@pytest.mark.parametrize("group", range(4))
+def test_fused_decode_exact_on_every_bf16_tie(group):
+    """The same rows through the fused decode kernel's own quantiser, two
+    tokens per call (K = 34816, so K * 2 fits the decode kernel)."""
+    K, N = 34816, 64
+    W, _ = inputs.make_case(4242, 1, K, N)
+    ref_packed, ref_gamma, _ = orc.pack_weights(W)
+    _, _, packed, gamma = gpu_pack(W)
+    mant = list(range(128 + 32 * group, 160 + 32 * group))
+    x = _tie_rows(mant, K)
+    ref_xq, ref_eta, ref_xsum = orc.quant_act(x)
+    for i in range(0, len(mant), 2):
+        xd = torch.from_numpy(x[i:i + 2]).cuda().to(torch.bfloat16)
+        y, (xq, eta, xsum) = bl.linear(xd, packed, gamma, N, out_dtype=torch.float32, want_quant=True,
+                                       weights_static=True)
+        np.testing.assert_array_equal(xq.cpu().numpy(), ref_xq[i:i + 2])
+        np.testing.assert_array_equal(eta.cpu().numpy(), ref_eta[i:i + 2])
+        np.testing.assert_array_equal(xsum.cpu().numpy(), ref_xsum[i:i + 2])
+        _, ref_y = orc.forward(ref_xq[i:i + 2], ref_eta[i:i + 2], ref_packed, ref_gamma, K, N)
+        np.testing.assert_array_equal(y.cpu().numpy().view(np.uint32), ref_y.view(np.uint32))
+
+
+def test_quantiser_tiny_rows_use_the_eta_floor():
+    """Rows with max |x| < 1e-5: eta is the 1e-5 floor (not a bf16 value), so
+    ties go through the IEEE quotient.  Both quantisers."""
+    K = 4096
+    rng = np.random.default_rng(11)
+    bits = rng.integers(0x3000, 0x3727, size=(2, K)).astype(np.uint32)  # bf16 in ~[4.7e-10, 9.9e-6]
+    x = ((bits << 16).view(np.float32) * np.where(rng.random((2, K)) < 0.5, -1, 1)).astype(np.float32)
+    assert np.abs(x).max() < 1e-5
+    ref_xq, ref_eta, ref_xsum = orc.quant_act(x)
+    xq, eta, xsum = gpu_quant(x, "bf16")
+    np.testing.assert_array_equal(xq.cpu().numpy(), ref_xq)
+    np.testing.assert_array_equal(eta.cpu().numpy(), ref_eta)
+    W, _ = inputs.make_case(4243, 1, K, 32)
+    _, _, packed, gamma = gpu_pack(W)
+    y, (xq2, eta2, xsum2) = bl.linear(torch.from_numpy(x).cuda().to(torch.bfloat16), packed, gamma, 32,
+                                      out_dtype=torch.float32, want_quant=True)
+    np.testing.assert_array_equal(xq2.cpu().numpy(), ref_xq)
+    np.testing.assert_array_equal(xsum2.cpu().numpy(), ref_xsum)
