@@ -181,10 +181,10 @@ bl_status bitlinear_forward(const int8_t* xq, const float* eta, const int32_t* x
  * Flag for bitlinear_forward_path and bitlinear_linear: the caller promises
  * that `packed` and `gamma` are not written by any work still pending on
  * `stream` (true for weights packed earlier and synchronised, the normal
- * inference case).  The decode kernel may then start streaming the packed
- * weights before the preceding kernel on the stream has finished
- * (programmatic dependent launch); activations are always read only after
- * it has finished.
+ * inference case).  The decode and tensor-core kernels may then start
+ * streaming the packed weights (and read gamma) before the preceding kernel
+ * on the stream has finished (programmatic dependent launch); activations
+ * are always read only after it has finished.
  */
 #define BL_FLAG_WEIGHTS_STATIC 1u
 
@@ -254,6 +254,20 @@ bl_status bitlinear_decode_shape(int64_t M, int64_t K, int64_t N, int fused, int
  * Errors: BL_ERR_INVALID_ARG for values outside those ranges.
  */
 bl_status bitlinear_set_decode_shape(int team_warps, int rows_per_block);
+
+/*
+ * Force the K split of the tensor-core kernel (BL_PATH_TCGEN05) for every
+ * later launch in this process: k_split in 1..8 CTAs per cluster, each
+ * accumulating its share of the K tiles of 128, the partial int32 tiles
+ * added in distributed shared memory; 0 leaves the choice to the library
+ * (the default: split only when the output tiles cannot fill the GPU).  The
+ * split is capped by the K tiles and by the partial tiles the first CTA can
+ * hold.  The pages have no counterpart; results are identical for every
+ * split (integer sums).  Not synchronised with launches in flight on other
+ * host threads.
+ * Errors: BL_ERR_INVALID_ARG for k_split outside 0..8.
+ */
+bl_status bitlinear_set_tc_split(int k_split);
 
 /* The path bitlinear_forward would pick for these sizes and pointers. */
 bl_path bitlinear_select_path(int64_t M, int64_t K, int64_t N,

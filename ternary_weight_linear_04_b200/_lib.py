@@ -36,6 +36,7 @@ SIGNATURES = {
     "bitlinear_device_error": (_I, [_P, _P]),
     "bitlinear_decode_shape": (_I, [_I64, _I64, _I64, _I, _P]),
     "bitlinear_set_decode_shape": (_I, [_I, _I]),
+    "bitlinear_set_tc_split": (_I, [_I]),
 }
 
 _lib = None

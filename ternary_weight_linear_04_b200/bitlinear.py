@@ -114,6 +114,12 @@ def decode_shape(M, K, N, fused=True):
     return dict(zip(DECODE_SHAPE_FIELDS, list(buf)))
 
 
+def set_tc_split(k_split=0):
+    """Force the K split (CTAs per cluster) of the tensor-core kernel for later
+    launches in this process (0 = the library's choice)."""
+    check(_lib.lib().bitlinear_set_tc_split(k_split), "bitlinear_set_tc_split")
+
+
 def set_decode_shape(team_warps=0, rows_per_block=0):
     """Force the decode kernel's team width and row-block height for later
     launches in this process (0 = the library's choice)."""

@@ -72,6 +72,32 @@ bl_status launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
   return launch_status();
 }
 
+// The same, as thread-block clusters of `cluster_z` CTAs along grid z.
+template <typename... KArgs, typename... Args>
+bl_status launch_pdl_cluster(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                             cudaStream_t st, unsigned cluster_z, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = 1;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = cluster_z;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    return BL_ERR_CUDA;
+  }
+  return launch_status();
+}
+
 // Once per device: is it an sm_100 part, and how many SMs does it have.
 struct DeviceInfo {
   int checked = 0;
@@ -333,10 +359,30 @@ bl_status launch_generic(const int8_t* xq, const float* eta, int64_t M, int64_t 
   return BL_OK;
 }
 
+// K split of the tensor-core kernel: when the output tiles cannot fill the
+// GPU (few tokens), CTAs split K in clusters of up to 8 and add their
+// partial tiles in distributed shared memory.  floor(SMs / tiles) splits
+// (the whole grid in one wave of one CTA per SM; measured faster than
+// filling both CTA slots of the small token tiles), at least two K tiles of
+// 128 per CTA, and no more partial tiles than CTA 0's stage memory holds.
+std::atomic<int> g_force_split{0};
+
+template <int BM>
+int tc_split(int64_t tiles, int64_t K, int sms) {
+  const int64_t KT = (K + bl::kTcBK - 1) / bl::kTcBK;
+  const int forced = g_force_split.load(std::memory_order_relaxed);
+  int64_t ks = forced > 0 ? forced : (tiles >= sms ? 1 : sms / tiles);
+  if (forced <= 0 && ks > KT / 2) ks = KT / 2;
+  if (ks > KT) ks = KT;
+  if (ks > bl::TcCfg<BM>::kMaxSplit) ks = bl::TcCfg<BM>::kMaxSplit;
+  if (ks < 1) ks = 1;
+  return static_cast<int>(ks);
+}
+
 template <int BM, typename OutT>
 bl_status launch_tc_bm(const int8_t* xq, const float* eta, const int32_t* xsum, int M, int K,
                        const uint8_t* packed, const float* gamma, int N, void* y, int32_t* y_int,
-                       cudaStream_t st) {
+                       int sms, int wstatic, cudaStream_t st) {
   using Cfg = bl::TcCfg<BM>;
   static int smem_done[kMaxDevices] = {0};
   auto kern = bl::k_gemm_tc<BM, OutT>;
@@ -349,19 +395,25 @@ bl_status launch_tc_bm(const int8_t* xq, const float* eta, const int32_t* xsum, 
     return BL_ERR_CUDA;
   dim3 grid((N + bl::kTcBN - 1) / bl::kTcBN, (M + BM - 1) / BM);
   if (grid.y > 65535) return BL_ERR_UNSUPPORTED;
-  return launch_pdl(kern, grid, dim3(bl::kTcThreads), Cfg::kSmem, st, tm_x, tm_w, eta, xsum, gamma,
-                    M, K, N, y, y_int);
+  const int ks = tc_split<BM>(grid.x * grid.y, K, sms);
+  if (ks <= 1)
+    return launch_pdl(kern, grid, dim3(bl::kTcThreads), Cfg::kSmem, st, tm_x, tm_w, eta, xsum,
+                      gamma, M, K, N, y, y_int, 1, wstatic);
+  grid.z = static_cast<unsigned>(ks);
+  return launch_pdl_cluster(kern, grid, dim3(bl::kTcThreads), Cfg::kSmem, st,
+                            static_cast<unsigned>(ks), tm_x, tm_w, eta, xsum, gamma, M, K, N, y,
+                            y_int, ks, wstatic);
 }
 
 template <typename OutT>
 bl_status launch_tc(const int8_t* xq, const float* eta, const int32_t* xsum, int M, int K,
                     const uint8_t* packed, const float* gamma, int N, void* y, int32_t* y_int,
-                    cudaStream_t st) {
-  if (M <= 16) return launch_tc_bm<16, OutT>(xq, eta, xsum, M, K, packed, gamma, N, y, y_int, st);
-  if (M <= 32) return launch_tc_bm<32, OutT>(xq, eta, xsum, M, K, packed, gamma, N, y, y_int, st);
-  if (M <= 64) return launch_tc_bm<64, OutT>(xq, eta, xsum, M, K, packed, gamma, N, y, y_int, st);
-  if (M <= 128) return launch_tc_bm<128, OutT>(xq, eta, xsum, M, K, packed, gamma, N, y, y_int, st);
-  return launch_tc_bm<256, OutT>(xq, eta, xsum, M, K, packed, gamma, N, y, y_int, st);
+                    int sms, int ws, cudaStream_t st) {
+  if (M <= 16) return launch_tc_bm<16, OutT>(xq, eta, xsum, M, K, packed, gamma, N, y, y_int, sms, ws, st);
+  if (M <= 32) return launch_tc_bm<32, OutT>(xq, eta, xsum, M, K, packed, gamma, N, y, y_int, sms, ws, st);
+  if (M <= 64) return launch_tc_bm<64, OutT>(xq, eta, xsum, M, K, packed, gamma, N, y, y_int, sms, ws, st);
+  if (M <= 128) return launch_tc_bm<128, OutT>(xq, eta, xsum, M, K, packed, gamma, N, y, y_int, sms, ws, st);
+  return launch_tc_bm<256, OutT>(xq, eta, xsum, M, K, packed, gamma, N, y, y_int, sms, ws, st);
 }
 
 bool fast_layout_ok(int64_t K, const void* xq, const void* packed, const void* y, const void* y_int) {
@@ -406,13 +458,15 @@ bl_status forward_impl(const int8_t* xq, const float* eta, const int32_t* xsum, 
                          : launch_decode<bl::DecNoFuse, __nv_bfloat16>(a, sms, s);
   }
   if (path == BL_PATH_TCGEN05) {
+    const int ws = (flags & BL_FLAG_WEIGHTS_STATIC) ? 1 : 0;
     if (!fast_layout_ok(K, xq, packed, y, y_int) || M > INT32_MAX / 2 || N > INT32_MAX / 2 ||
         K > (1 << 30))
       return BL_ERR_UNSUPPORTED;
     return ydt == BL_F32
-               ? launch_tc<float>(xq, eta, xsum, (int)M, (int)K, packed, gamma, (int)N, y, y_int, s)
+               ? launch_tc<float>(xq, eta, xsum, (int)M, (int)K, packed, gamma, (int)N, y, y_int,
+                                  sms, ws, s)
                : launch_tc<__nv_bfloat16>(xq, eta, xsum, (int)M, (int)K, packed, gamma, (int)N, y,
-                                          y_int, s);
+                                          y_int, sms, ws, s);
   }
   return ydt == BL_F32
              ? launch_generic<float>(xq, eta, M, K, packed, gamma, N, y, y_int, sms, s)
@@ -453,6 +507,12 @@ bl_status bitlinear_decode_shape(int64_t M, int64_t K, int64_t N, int fused, int
   shape[7] = g.stages;
   shape[8] = g.x_staged;
   shape[9] = static_cast<int32_t>(g.smem);
+  return BL_OK;
+}
+
+bl_status bitlinear_set_tc_split(int k_split) {
+  if (k_split < 0 || k_split > 8) return BL_ERR_INVALID_ARG;
+  g_force_split.store(k_split, std::memory_order_relaxed);
   return BL_OK;
 }
 

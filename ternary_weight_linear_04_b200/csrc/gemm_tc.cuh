@@ -16,19 +16,32 @@
 //
 // Tile: 128 output features (the MMA's M, operand A = weights) by BM tokens
 // (the MMA's N, operand B = activations), K in stages of 128.  Per stage:
-//   * warp 0 (one thread) issues two TMA loads: the BM x 128 int8 activation
-//     tile (128-byte swizzle, K-major) and the 128 x 32-byte packed weight
-//     tile;
+//   * warp 0 issues two TMA loads: lane 1 the 128 x 32-byte packed weight
+//     tile, lane 0 the BM x 128 int8 activation tile (128-byte swizzle,
+//     K-major).  When the caller declares the weights static, the packed
+//     tiles of the first S stages are requested before griddepcontrol.wait,
+//     overlapping the preceding kernel;
 //   * warps 2-9 expand the packed codes (each thread: half of one row's 32
 //     bytes, i.e. 64 codes) to bytes in natural k order, directly in the
 //     128-byte swizzled K-major layout the MMA reads, then fence the
 //     generic->async proxy and arrive (one arrival per warp);
 //   * warp 1 (one thread) issues four 128 x BM x 32 MMAs and commits the
-//     stage back to the producer.
+//     stage back (one commit per stage: the MMA thread's issue rate bounds
+//     the small token tiles).
 // After the K loop warps 2-9 read the accumulator (one TMEM lane = one
 // output feature; the two warps of a lane quarter split the token columns),
-// subtract xsum, rescale and store.  Every barrier wait is bounded (see
-// common.cuh).  No cluster, no multicast.
+// subtract xsum, rescale and store.
+//
+// Split K (few tokens, so fewer tiles than SMs): the launch groups
+// `ksplit` CTAs along K into a thread-block cluster; CTA r accumulates K
+// tiles [KT*r/ksplit, KT*(r+1)/ksplit) in its own TMEM.  After a cluster
+// barrier (every MMA of the cluster done, so the stage memory of CTA 0 is
+// free) CTAs 1.. store their int32 partial tiles into CTA 0's stage memory
+// through distributed shared memory; after a second barrier CTA 0 adds
+// them to its own accumulator and runs the epilogue.  Integer sums, so the
+// result does not depend on the split.  Every barrier wait is bounded (see
+// common.cuh); the cluster barriers count exited threads as arrived.  No
+// multicast.
 #pragma once
 
 #include <cuda.h>
@@ -44,33 +57,43 @@ constexpr int kTcThreads = 32 * (2 + kTcUnpackWarps);
 
 template <int BM>
 struct TcCfg {
-  static constexpr int kStages = BM >= 256 ? 4 : (BM >= 128 ? 5 : 6);
+  // few stages for the small token tiles: two CTAs fit per SM
+  static constexpr int kStages = BM >= 256 ? 4 : (BM >= 128 ? 5 : (BM >= 64 ? 6 : 4));
   static constexpr int kABytes = kTcBN * kTcBK;        // unpacked weights
   static constexpr int kBBytes = BM * kTcBK;           // activations
   static constexpr int kPBytes = kTcBN * (kTcBK / 4);  // packed weights
+  static constexpr size_t kStageRegion =
+      static_cast<size_t>(kStages) * (kABytes + kBBytes + kPBytes);
+  // largest split whose partial tiles fit in CTA 0's stage memory
+  static constexpr int kMaxSplit =
+      1 + static_cast<int>(kStageRegion / (static_cast<size_t>(kTcBN) * BM * 4)) > 8
+          ? 8
+          : 1 + static_cast<int>(kStageRegion / (static_cast<size_t>(kTcBN) * BM * 4));
   static constexpr int kTmemCols = BM < 32 ? 32 : BM;
-  static constexpr int kBarBytes = 8 * (3 * kStages + 1) + 16 + 8 * BM;
-  static constexpr size_t kSmem =
-      1024 + static_cast<size_t>(kStages) * (kABytes + kBBytes + kPBytes) + kBarBytes;
+  static constexpr int kBarBytes = 8 * (4 * kStages + 1) + 16 + 8 * BM;
+  static constexpr size_t kSmem = 1024 + kStageRegion + kBarBytes;
+  static_assert(kSmem <= 227 * 1024, "shared memory per CTA");
+  static_assert(BM > 32 || kSmem <= 113 * 1024, "two CTAs per SM for the small token tiles");
 };
 
 template <int BM, typename OutT>
-__global__ void __launch_bounds__(kTcThreads, 1)
+__global__ void __launch_bounds__(kTcThreads, BM <= 32 ? 2 : 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
               const float* __restrict__ eta, const int32_t* __restrict__ xsum,
               const float* __restrict__ gamma_p, int M, int K, int N, void* __restrict__ y,
-              int32_t* __restrict__ y_int) {
+              int32_t* __restrict__ y_int, int ksplit, int wstatic) {
   using Cfg = TcCfg<BM>;
   constexpr int S = Cfg::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint8_t* sA = base;
-  uint8_t* sB = sA + S * Cfg::kABytes;
-  uint8_t* sP = sB + S * Cfg::kBBytes;
-  uint64_t* full_tma = reinterpret_cast<uint64_t*>(sP + S * Cfg::kPBytes);
-  uint64_t* full_a = full_tma + S;
-  uint64_t* empty = full_a + S;
+  uint8_t* sA = base;                    // [S] unpacked weights
+  uint8_t* sB = sA + S * Cfg::kABytes;   // [S] activations
+  uint8_t* sP = sB + S * Cfg::kBBytes;   // [S] packed weights
+  uint64_t* full_a = reinterpret_cast<uint64_t*>(sP + S * Cfg::kPBytes);  // unpacked (8 warps)
+  uint64_t* full_p = full_a + S;  // packed weight tile in
+  uint64_t* full_b = full_p + S;  // activation tile in
+  uint64_t* empty = full_b + S;   // the MMA is done with the stage
   uint64_t* accum_full = empty + S;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum_full + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -82,11 +105,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int n0 = blockIdx.x * kTcBN;
   const int m0 = blockIdx.y * BM;
   const int KT = (K + kTcBK - 1) / kTcBK;
+  const int zr = ksplit > 1 ? static_cast<int>(cluster_ctarank()) : 0;
+  const int kt0 = static_cast<int>(static_cast<int64_t>(KT) * zr / ksplit);
+  const int nkt = static_cast<int>(static_cast<int64_t>(KT) * (zr + 1) / ksplit) - kt0;  // >= 1
 
+  auto issue_p = [&](int i) {  // packed weight tile i of this CTA's K range
+    const int s = i % S;
+    mbar_arrive_expect_tx(full_p + s, Cfg::kPBytes);
+    tma_load_2d(sP + s * Cfg::kPBytes, &tm_w, full_p + s, (kt0 + i) * (kTcBK / 4), n0);
+  };
+  const int p_first = nkt < S ? nkt : S;
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(full_tma + s, 1);
       mbar_init(full_a + s, kTcUnpackWarps);
+      mbar_init(full_p + s, 1);
+      mbar_init(full_b + s, 1);
       mbar_init(empty + s, 1);
     }
     mbar_init(accum_full, 1);
@@ -94,6 +127,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     mbar_init_fence();
     tma_prefetch_desc(&tm_x);
     tma_prefetch_desc(&tm_w);
+    if (wstatic)
+      for (int i = 0; i < p_first; ++i) issue_p(i);  // not written by the preceding kernel
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, Cfg::kTmemCols);
@@ -113,65 +148,76 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_d = *tmem_slot;
+  bool epi_ok = false;  // unpack warps: the accumulator is complete
 
   if (warp == 0) {
-    // ---------------- TMA producer
+    // ---------------- TMA producers: lane 0 activations, lane 1 packed weights
     if (lane == 0) {
-      for (int kt = 0; kt < KT; ++kt) {
-        const int s = kt % S;
-        const uint32_t round = static_cast<uint32_t>(kt / S);
-        if (kt >= S && !mbar_wait(empty + s, (round - 1) & 1u, abort_flag)) break;
-        mbar_arrive_expect_tx(full_tma + s, Cfg::kBBytes + Cfg::kPBytes);
-        tma_load_2d(sB + s * Cfg::kBBytes, &tm_x, full_tma + s, kt * kTcBK, m0);
-        tma_load_2d(sP + s * Cfg::kPBytes, &tm_w, full_tma + s, kt * (kTcBK / 4), n0);
+      for (int i = 0; i < nkt; ++i) {
+        const int s = i % S;
+        if (i >= S && !mbar_wait(empty + s, static_cast<uint32_t>(i / S - 1) & 1u, abort_flag)) break;
+        mbar_arrive_expect_tx(full_b + s, Cfg::kBBytes);
+        tma_load_2d(sB + s * Cfg::kBBytes, &tm_x, full_b + s, (kt0 + i) * kTcBK, m0);
+      }
+    } else if (lane == 1) {
+      if (!wstatic)
+        for (int i = 0; i < p_first; ++i) issue_p(i);
+      for (int i = S; i < nkt; ++i) {
+        if (!mbar_wait(empty + i % S, static_cast<uint32_t>(i / S - 1) & 1u, abort_flag)) break;
+        issue_p(i);
       }
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = make_idesc_i8_u8s8(kTcBN, BM);
+      // Descriptors of stage 0, advanced by adding to the start-address field
+      // (address >> 4 in the low bits; every stage address stays below 2^18,
+      // so the field never carries): +S_bytes/16 per stage, +2 per K step of
+      // 32 bytes.  Keeps the single issuing thread's work per stage short.
+      const uint64_t a_desc0 = make_sw128_kmajor_desc(smem_u32(sA));
+      const uint64_t b_desc0 = make_sw128_kmajor_desc(smem_u32(sB));
       bool ok = true;
-      for (int kt = 0; kt < KT; ++kt) {
-        const int s = kt % S;
-        const uint32_t par = static_cast<uint32_t>(kt / S) & 1u;
-        ok = mbar_wait(full_tma + s, par, abort_flag) && mbar_wait(full_a + s, par, abort_flag);
+      for (int i = 0; i < nkt; ++i) {
+        const int s = i % S;
+        const uint32_t par = static_cast<uint32_t>(i / S) & 1u;
+        ok = mbar_wait(full_b + s, par, abort_flag) && mbar_wait(full_a + s, par, abort_flag);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t a0 = smem_u32(sA + s * Cfg::kABytes);
-        const uint32_t b0 = smem_u32(sB + s * Cfg::kBBytes);
+        const uint64_t ad = a_desc0 + static_cast<uint64_t>(s * (Cfg::kABytes >> 4));
+        const uint64_t bd = b_desc0 + static_cast<uint64_t>(s * (Cfg::kBBytes >> 4));
+        tc_mma_i8_ss(tmem_d, ad, bd, idesc, i != 0 ? 1u : 0u);
 #pragma unroll
-        for (int kk = 0; kk < kTcBK / 32; ++kk)
-          tc_mma_i8_ss(tmem_d, make_sw128_kmajor_desc(a0 + 32 * kk),
-                       make_sw128_kmajor_desc(b0 + 32 * kk), idesc, (kt | kk) != 0 ? 1u : 0u);
+        for (int kk = 1; kk < kTcBK / 32; ++kk)
+          tc_mma_i8_ss(tmem_d, ad + 2 * kk, bd + 2 * kk, idesc, 1u);
         tc_commit(empty + s);
       }
       if (ok) tc_commit(accum_full);
     }
   } else {
     // ---------------- unpack, then epilogue (warps 2..9)
-    const int u = warp - 2;          // 0..7
-    const int q = warp & 3;          // TMEM lane quarter this warp may access
-    const int row = q * 32 + lane;   // weight row (output feature) in the tile
-    const int half = u >> 2;         // which half of the row's 32 packed bytes
-    const int r8 = row & 7;
-    uint8_t* a_row = sA + (row >> 3) * 1024 + r8 * 128;
+    const int u = warp - 2;            // 0..7
+    const int urow = (warp & 3) * 32 + lane;  // weight row (output feature) in the tile
+    const int uhalf = u >> 2;          // which half of the row's 32 packed bytes
+    const int r8 = urow & 7;
+    uint8_t* a_row = sA + (urow >> 3) * 1024 + r8 * 128;
     bool ok = true;
-    for (int kt = 0; kt < KT; ++kt) {
-      const int s = kt % S;
-      const uint32_t par = static_cast<uint32_t>(kt / S) & 1u;
-      ok = __all_sync(0xFFFFFFFFu, mbar_wait(full_tma + s, par, abort_flag));
+    for (int i = 0; i < nkt; ++i) {
+      const int s = i % S;
+      // the packed tile is in (its load waited for the MMA to free the stage)
+      ok = __all_sync(0xFFFFFFFFu, mbar_wait(full_p + s, static_cast<uint32_t>(i / S) & 1u, abort_flag));
       if (!ok) break;
-      const uint4 p = *reinterpret_cast<const uint4*>(sP + s * Cfg::kPBytes + row * 32 + half * 16);
+      const uint4 p = *reinterpret_cast<const uint4*>(sP + s * Cfg::kPBytes + urow * 32 + uhalf * 16);
       const uint32_t pw[4] = {p.x, p.y, p.z, p.w};
       uint8_t* dst = a_row + s * Cfg::kABytes;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int c = half * 4 + i;  // 16-byte chunk of the 128-byte row
+      for (int wi = 0; wi < 4; ++wi) {
+        const int c = uhalf * 4 + wi;  // 16-byte chunk of the 128-byte row
         // word c holds the codes of k = 16c .. 16c+15; byte b bits 2j = k 16c+4b+j
-        const uint32_t t0 = pw[i] & 0x03030303u;
-        const uint32_t t1 = (pw[i] >> 2) & 0x03030303u;
-        const uint32_t t2 = (pw[i] >> 4) & 0x03030303u;
-        const uint32_t t3 = (pw[i] >> 6) & 0x03030303u;
+        const uint32_t t0 = pw[wi] & 0x03030303u;
+        const uint32_t t1 = (pw[wi] >> 2) & 0x03030303u;
+        const uint32_t t2 = (pw[wi] >> 4) & 0x03030303u;
+        const uint32_t t3 = (pw[wi] >> 6) & 0x03030303u;
         uint32_t o0, o1, o2, o3;
         transpose4x4_bytes(t0, t1, t2, t3, o0, o1, o2, o3);  // natural k order
         *reinterpret_cast<uint4*>(dst + ((c ^ r8) << 4)) = make_uint4(o0, o1, o2, o3);
@@ -181,28 +227,68 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (lane == 0) mbar_arrive(full_a + s);
     }
     if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait(accum_full, 0, abort_flag));
-    if (ok) {
-      tc_fence_after();
-      const int n = n0 + row;
-      const uint32_t t_row = tmem_d + (static_cast<uint32_t>(q * 32) << 16);
-      constexpr int kColsPerWarp = BM < 32 ? 16 : BM / 2;  // two warps per lane quarter
-      const int col0 = (BM < 32) ? 0 : half * kColsPerWarp;
-      if (!(BM < 32 && half == 1)) {
+    epi_ok = ok;
+  }
+
+  // ---------------- epilogue (warps 2..9): one TMEM lane = one output feature
+  const bool epi_warp = warp >= 2;
+  const int q = warp & 3;
+  const int row = q * 32 + lane;
+  const int half = (warp - 2) >> 2;
+  constexpr int kColsPerWarp = BM < 32 ? 16 : BM / 2;  // two warps per lane quarter
+  const int col0 = (BM < 32) ? 0 : half * kColsPerWarp;
+  const bool epi_cols = epi_warp && !(BM < 32 && half == 1);
+  const uint32_t t_row = tmem_d + (static_cast<uint32_t>(q * 32) << 16);
+  // CTA 0's stage memory receives the partial tiles of CTAs 1..ksplit-1:
+  // slot r-1, [128 rows][BM columns] int32
+  int32_t* part = reinterpret_cast<int32_t*>(sA);
+  if (ksplit > 1) {
+    __syncwarp();  // the cluster barrier is warp-aligned: reconverge after the role branches
+    tc_fence_before();
+    cluster_sync_all();  // every MMA of the cluster is done; CTA 0's stages are free
+    tc_fence_after();
+    if (zr != 0 && epi_cols && epi_ok) {
+      int32_t* slot = part + static_cast<size_t>(zr - 1) * kTcBN * BM + static_cast<size_t>(row) * BM;
 #pragma unroll 1
-        for (int cc = col0; cc < col0 + kColsPerWarp; cc += 16) {
-          uint32_t v[16];
-          tmem_ld_32x32b_x16(t_row + cc, v);
-          tmem_ld_wait();
+      for (int cc = col0; cc < col0 + kColsPerWarp; cc += 16) {
+        uint32_t v[16];
+        tmem_ld_32x32b_x16(t_row + cc, v);
+        tmem_ld_wait();
+        const uint32_t dst = cluster_map(slot + cc, 0);
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int m = m0 + cc + j;
-            if (m < M && n < N) {
-              const int32_t yi = static_cast<int32_t>(v[j]) - s_xsum[cc + j];
-              const int64_t o = static_cast<int64_t>(m) * N + n;
-              store_out<OutT>(y, o, rescale(yi, s_scale[cc + j]));
-              if (y_int) y_int[o] = yi;
-            }
-          }
+        for (int j = 0; j < 16; j += 4) st_cluster_v4(dst + 4 * j, v[j], v[j + 1], v[j + 2], v[j + 3]);
+      }
+    }
+    __syncwarp();
+    cluster_sync_all();  // the partial tiles are in CTA 0
+  }
+  if (zr == 0 && epi_cols && epi_ok) {
+    tc_fence_after();
+    const int n = n0 + row;
+#pragma unroll 1
+    for (int cc = col0; cc < col0 + kColsPerWarp; cc += 16) {
+      uint32_t v[16];
+      tmem_ld_32x32b_x16(t_row + cc, v);
+      tmem_ld_wait();
+      for (int r = 1; r < ksplit; ++r) {
+        const int32_t* src = part + static_cast<size_t>(r - 1) * kTcBN * BM + static_cast<size_t>(row) * BM + cc;
+#pragma unroll
+        for (int j = 0; j < 16; j += 4) {
+          const int4 t = *reinterpret_cast<const int4*>(src + j);
+          v[j] += static_cast<uint32_t>(t.x);
+          v[j + 1] += static_cast<uint32_t>(t.y);
+          v[j + 2] += static_cast<uint32_t>(t.z);
+          v[j + 3] += static_cast<uint32_t>(t.w);
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int m = m0 + cc + j;
+        if (m < M && n < N) {
+          const int32_t yi = static_cast<int32_t>(v[j]) - s_xsum[cc + j];
+          const int64_t o = static_cast<int64_t>(m) * N + n;
+          store_out<OutT>(y, o, rescale(yi, s_scale[cc + j]));
+          if (y_int) y_int[o] = yi;
         }
       }
     }

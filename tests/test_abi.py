@@ -91,6 +91,9 @@ def test_bad_arguments_are_rejected_without_a_launch(L):
     assert L.bitlinear_set_decode_shape(0, 3) == _lib.BL_ERR_INVALID_ARG
     assert L.bitlinear_set_decode_shape(0, 32) == _lib.BL_ERR_INVALID_ARG
     assert L.bitlinear_set_decode_shape(0, 0) == _lib.BL_OK
+    assert L.bitlinear_set_tc_split(-1) == _lib.BL_ERR_INVALID_ARG
+    assert L.bitlinear_set_tc_split(9) == _lib.BL_ERR_INVALID_ARG
+    assert L.bitlinear_set_tc_split(0) == _lib.BL_OK
 
 
 def test_path_selection_is_host_logic(L):

@@ -102,6 +102,31 @@ def test_paths_agree_with_oracle(path, M, K, N, out):
     check_layer(W, x, "bf16", out, path=path)
 
 
+@pytest.fixture
+def forced_split():
+    yield bl.set_tc_split
+    bl.set_tc_split(0)
+
+
+@pytest.mark.parametrize("M", [1, 5, 16, 17, 32, 33, 64, 65, 128])
+@pytest.mark.parametrize("ks", [2, 3, 5, 8])
+def test_tcgen05_split_k_clusters(forced_split, M, ks):
+    """K split across a cluster of ks CTAs, partial tiles added in CTA 0's
+    shared memory: every token tile width, uneven K shares (K = 1600 = 12.5
+    tiles of 128, so the last tile is ragged and the shares differ), N with a
+    partial feature tile."""
+    forced_split(ks)
+    W, x = inputs.make_case(3100 + 7 * M + ks, M, 1600, 389, act_dtype="bf16")
+    check_layer(W, x, "bf16", "bf16", path="tcgen05")
+
+
+@pytest.mark.parametrize("M,K,N", [(16, 3200, 8640), (16, 8640, 3200), (8, 8192, 1000), (32, 28672, 512)])
+def test_tcgen05_auto_split_decode_shapes(M, K, N):
+    """The library's own split choice on decode-sized batches."""
+    W, x = inputs.make_case(3300 + M + K, M, K, N, act_dtype="bf16")
+    check_layer(W, x, "bf16", "bf16", path="tcgen05")
+
+
 @pytest.mark.parametrize("M", [9, 16, 17, 31, 32, 33, 64, 65, 127, 128, 129, 200, 256, 257, 300])
 def test_tcgen05_token_tiles_and_tails(M):
     """Every token-tile width (16..256) plus ragged tails in M, N and K
