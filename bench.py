@@ -198,12 +198,13 @@ def run_ours(args, world, rank, local):
     M = args.m
     mats = []
     for j, mat in enumerate(wl.matrices):
-        W, x = inputs.make_matrix_inputs(wl, j, m_max=M)
+        W, x = inputs.make_matrix_inputs(wl, j, m_max=max(M, 64))  # 64 rows for the M sweep
         Wd = torch.from_numpy(W).to(dev)
         with torch.cuda.stream(stream):
             packed, gamma = bl.pack_weights(Wd, stream=stream)
-        xd = torch.from_numpy(x).to(dev).to(torch.bfloat16)
-        mats.append(dict(K=mat.K, N=mat.N, W=Wd, packed=packed, gamma=gamma, x=xd,
+        x_all = torch.from_numpy(x).to(dev).to(torch.bfloat16)
+        xd = x_all[:M]
+        mats.append(dict(K=mat.K, N=mat.N, W=Wd, packed=packed, gamma=gamma, x=xd, x_all=x_all,
                          xq=torch.empty((M, mat.K), dtype=torch.int8, device=dev),
                          eta=torch.empty(M, dtype=torch.float32, device=dev),
                          xsum=torch.empty(M, dtype=torch.int32, device=dev),
@@ -291,7 +292,8 @@ def run_ours(args, world, rank, local):
            "roofline": roofline, "gpu_launches": launches,
            "clocks": clk.summary()}
 
-    sections = set(args.sections.split(",")) if args.sections else {"e2e", "prefill", "pack"}
+    sections = (set(args.sections.split(",")) if args.sections else
+                {"e2e", "prefill", "pack", "sweep", "layer70b", "crossover"})
     if args.quick:
         sections = set()
     if "e2e" in sections:
@@ -300,6 +302,16 @@ def run_ours(args, world, rank, local):
         out["prefill"] = run_prefill(args, dev, stream, peaks, peak_src, world)
     if "pack" in sections:
         out["pack"] = run_pack(mats, stream, world)
+    if "sweep" in sections:
+        out["decode_sweep"] = run_sweep(mats, stream, world, peaks)
+    if "layer70b" in sections or "crossover" in sections:
+        for m in mats:  # free the headline workload's copies first
+            m["copies"] = m["copies"][:1]
+        torch.cuda.empty_cache()
+    if "layer70b" in sections:
+        out["layer_70b"] = run_layer70b(dev, stream, world, peaks, l2)
+    if "crossover" in sections:
+        out["crossover"] = run_crossover(dev, stream, world, peaks, l2)
     if (rank == 0) and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = run_cpu_baseline(args.cpu_seconds)
     return out
@@ -401,6 +413,163 @@ def run_prefill(args, dev, stream, peaks, peak_src, world):
             "peak_source": "%s bf16_tflops (burst) x %.0f nominal int8:bf16 ratio" % (peak_src, INT8_PER_BF16),
             "addsub_ops_needed_frac": "nnz(W~)/(N*K) of the dense ops (about 0.69)",
             "quant_us": round(tq * 1e6, 2), "quant_gbs": round(qbytes / tq / 1e9, 1)}
+
+
+def time_linear_step(mats, M, stream, world, min_seconds=0.25, xkey="x"):
+    """Seconds per step of one bitlinear_linear call per matrix (static
+    weights), CUDA graph over every rotating packed copy, max over ranks.
+    mats: dicts with K, N, copies [(packed, gamma)], m[xkey] (>= M rows, bf16)."""
+    from ternary_weight_linear_04_b200 import _lib
+    L = _lib.lib()
+    P = ctypes.c_void_p
+    dev = mats[0][xkey].device
+    sptr = ctypes.c_void_p(stream.cuda_stream)
+    bufs = []
+    for m in mats:
+        bufs.append(dict(x=m[xkey][:M].contiguous(),
+                         y=torch.empty((M, m["N"]), dtype=torch.bfloat16, device=dev),
+                         xq=torch.empty((M, m["K"]), dtype=torch.int8, device=dev),
+                         eta=torch.empty(M, dtype=torch.float32, device=dev),
+                         xsum=torch.empty(M, dtype=torch.int32, device=dev)))
+
+    def call(m, b, c):
+        pk, g = m["copies"][c]
+        a = (P(b["x"].data_ptr()), _lib.BL_BF16, M, m["K"], P(pk.data_ptr()), P(g.data_ptr()), m["N"],
+             P(b["y"].data_ptr()), _lib.BL_BF16, P(b["xq"].data_ptr()), P(b["eta"].data_ptr()),
+             P(b["xsum"].data_ptr()), None, _lib.BL_FLAG_WEIGHTS_STATIC, sptr)
+        return lambda: _chk(L.bitlinear_linear(*a), "linear")
+
+    copies = len(mats[0]["copies"])
+    calls = [call(m, b, c) for c in range(copies) for m, b in zip(mats, bufs)]
+    with torch.cuda.stream(stream):
+        for fn in calls:
+            fn()
+    torch.cuda.synchronize()
+    g = Capture(calls, stream)
+    with torch.cuda.stream(stream):
+        g.replay()
+    torch.cuda.synchronize()
+    t1 = timed(lambda: g.replay(), stream, world)
+    reps = max(3, int(min_seconds / max(t1, 1e-6)))
+    t = timed(lambda: [g.replay() for _ in range(reps)], stream, world)
+    t = max_over_ranks(t, world)
+    return t / (reps * copies)
+
+
+def make_bench_mats(wl_name, M, dev, stream, l2, copies=None):
+    """Packed matrices of a workload (+ rotating copies past 3x L2) and its
+    activations (M rows)."""
+    from ternary_weight_linear_04_b200 import inputs
+    from ternary_weight_linear_04_b200 import bitlinear as bl
+    wl = inputs.WORKLOADS[wl_name]
+    mats = []
+    for j, mat in enumerate(wl.matrices):
+        W, x = inputs.make_matrix_inputs(wl, j, m_max=M)
+        with torch.cuda.stream(stream):
+            Wd = torch.from_numpy(W).to(dev)
+            packed, gamma = bl.pack_weights(Wd, stream=stream)
+        torch.cuda.synchronize()
+        del Wd, W
+        mats.append(dict(K=mat.K, N=mat.N, name=mat.name, packed=packed, gamma=gamma,
+                         x=torch.from_numpy(x).to(dev).to(torch.bfloat16)))
+    wbytes = sum(m["N"] * ((m["K"] + 3) // 4) for m in mats)
+    if copies is None:
+        copies = max(2, int(np.ceil(3 * l2 / wbytes)))
+    for m in mats:
+        m["copies"] = [(m["packed"], m["gamma"])] + [(m["packed"].clone(), m["gamma"].clone())
+                                                     for _ in range(copies - 1)]
+    torch.cuda.synchronize()
+    return mats, copies, wbytes
+
+
+def run_sweep(mats, stream, world, peaks, Ms=(4, 8, 16, 32, 64)):
+    """decode_3b at the other batch sizes SURVEY-style: GB/s against HBM."""
+    from ternary_weight_linear_04_b200 import bitlinear as bl
+    hbm = float(peaks["hbm_gbs"])
+    rows = []
+    for M in Ms:
+        t = time_linear_step(mats, M, stream, world, xkey="x_all")
+        b = sum(linear_bytes(M, m["K"], m["N"]) for m in mats)
+        paths = ["gemv (fused)" if bl.fused_decode_ok(M, m["K"]) else
+                 bl.select_path(M, m["K"], m["N"], m["x_all"], m["packed"], m["x_all"]) for m in mats]
+        rows.append({"M": M, "us_per_step": round(t * 1e6, 2), "gbs": round(b / t / 1e9, 1),
+                     "frac": round(b / t / 1e9 / hbm, 4), "paths": paths})
+    return {"workload": "decode_3b: K=3200->N=8640 and K=8640->N=3200, bf16 in/out",
+            "step": "one bitlinear_linear per matrix (quantise + accumulate + rescale)",
+            "rows": rows}
+
+
+def run_layer70b(dev, stream, world, peaks, l2):
+    """One 70B-class decoder layer's 7 projections as 7 calls, M = 1 and 32."""
+    hbm = float(peaks["hbm_gbs"])
+    mats, copies, wbytes = make_bench_mats("layer_70b", 32, dev, stream, l2)
+    rows = []
+    for M in (1, 32):
+        t = time_linear_step(mats, M, stream, world)
+        b = sum(linear_bytes(M, m["K"], m["N"]) for m in mats)
+        rows.append({"M": M, "us_per_layer": round(t * 1e6, 2), "gbs": round(b / t / 1e9, 1),
+                     "frac": round(b / t / 1e9 / hbm, 4)})
+    del mats
+    torch.cuda.empty_cache()
+    return {"workload": "layer_70b: Wq 8192^2, Wk/Wv 8192x1024, Wo 8192^2, gate/up 8192x28672, "
+                        "down 28672x8192; 7 bitlinear_linear calls per step",
+            "packed_bytes_per_layer": wbytes, "copies": copies, "rows": rows}
+
+
+def run_crossover(dev, stream, world, peaks, l2):
+    """8192x28672, Laplace weights, Student-t(3) activations with 1% x50
+    outlier channels: both accumulate paths across M; the crossover is the
+    smallest M at which the tensor-core path is the faster one."""
+    from ternary_weight_linear_04_b200 import _lib
+    from ternary_weight_linear_04_b200 import bitlinear as bl
+    mats, copies, wbytes = make_bench_mats("outlier_sweep", 2048, dev, stream, l2)
+    m = mats[0]
+    K, N = m["K"], m["N"]
+    hbm = float(peaks["hbm_gbs"])
+    peak_t = float(peaks["bf16_tflops"]) * INT8_PER_BF16
+    L = _lib.lib()
+    P = ctypes.c_void_p
+    sptr = ctypes.c_void_p(stream.cuda_stream)
+    rows, cross = [], None
+    for M in (1, 2, 4, 8, 64, 256, 2048):
+        xq, eta, xsum = bl.quant_act(m["x"][:M].contiguous(), stream=stream)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        torch.cuda.synchronize()
+        row = {"M": M}
+        for path in (("gemv", "tcgen05") if M <= 4 else ("tcgen05",)):
+            calls = []
+            for c in range(copies):
+                pk, g = m["copies"][c]
+                a = (P(xq.data_ptr()), P(eta.data_ptr()), P(xsum.data_ptr()), M, K, P(pk.data_ptr()),
+                     P(g.data_ptr()), N, P(y.data_ptr()), _lib.BL_BF16, None, bl.PATHS[path],
+                     _lib.BL_FLAG_WEIGHTS_STATIC, sptr)
+                calls.append(lambda a=a: _chk(L.bitlinear_forward_path(*a), path))
+            with torch.cuda.stream(stream):
+                for fn in calls:
+                    fn()
+            torch.cuda.synchronize()
+            gr = Capture(calls, stream)
+            with torch.cuda.stream(stream):
+                gr.replay()
+            torch.cuda.synchronize()
+            reps = 20 if M <= 256 else 3
+            t = max_over_ranks(timed(lambda: [gr.replay() for _ in range(reps)], stream, world),
+                               world) / (reps * copies)
+            b = linear_bytes(M, K, N, in_bytes=1)
+            row[path] = {"us": round(t * 1e6, 2), "gbs": round(b / t / 1e9, 1),
+                         "hbm_frac": round(b / t / 1e9 / hbm, 4),
+                         "tops": round(2.0 * M * N * K / t / 1e12, 1),
+                         "tensor_frac": round(2.0 * M * N * K / t / 1e12 / peak_t, 4)}
+        if cross is None and "gemv" in row and row["tcgen05"]["us"] <= row["gemv"]["us"]:
+            cross = M
+        rows.append(row)
+    del mats
+    torch.cuda.empty_cache()
+    return {"workload": "outlier_sweep: K=8192, N=28672, Laplace(0,0.02) W, Student-t(3) x with "
+                        "1%% x50 channels; accumulate kernel only (x~ given)",
+            "rows": rows,
+            "crossover_M": cross if cross is not None else "above 4 (the CUDA-core decode path "
+                                                           "takes M <= 4 and is faster there)"}
 
 
 def run_pack(mats, stream, world):
@@ -516,7 +685,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--m", type=int, default=1, help="tokens per step (decode batch)")
     ap.add_argument("--quick", action="store_true", help="headline only (no e2e/prefill/pack)")
-    ap.add_argument("--sections", default="", help="comma list of extra sections: e2e,prefill,pack")
+    ap.add_argument("--sections", default="",
+                    help="comma list of extra sections: e2e,prefill,pack,sweep,layer70b,crossover")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     args = ap.parse_args()

@@ -7,6 +7,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <cmath>
 #include <cstdint>
 #include <cstring>
 #include <atomic>
@@ -191,6 +192,10 @@ bool make_tmap_u8(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t col
 // largest of (instructions / 4 issue slots, dp4a / 2 per cycle, shared
 // memory wavefronts, and 2 x one warp's own instruction stream), with the
 // padding words (32*G*nwj >= K/16) and padding rows (blocks of RB) counted.
+// When the CTA's rows do not fit the ring (the weights stream while the
+// kernel runs), the stages must also keep enough copies in flight and
+// enough warps busy: a stage holds whole blocks, only the teams owning
+// them work on it, and `stages` stages cover the load latency.
 struct DecGeom {
   int G = 1, teams = 16, nwj = 1, RB = 1;
   int rows_per_cta = 1, grid = 1, bpc = 1, stages = 1, x_staged = 0;
@@ -201,6 +206,7 @@ constexpr size_t kDecTwoCtaSmem = 113 * 1024;  // two CTAs per SM (228 KB less 1
 constexpr size_t kDecMaxSmem = 227 * 1024;
 constexpr int64_t kDecRingBytes = 64 * 1024;
 constexpr int64_t kDecStageTarget = 32 * 1024;
+constexpr double kDecLoadLatency = 2000.0;  // cycles from a stage's copy request to its arrival
 
 inline bool rb_allowed(int MT, int RB) { return RB * MT <= 16; }
 
@@ -243,8 +249,32 @@ bool decode_geometry(int MT, int64_t M, int64_t K, int64_t N, int sms, int64_t x
       // shared memory: slots + ring of at least one block + tail
       const int64_t slots = static_cast<int64_t>(MT) * 32 * G * nwj * 16;
       const int64_t blk = RB * P;
-      if (slots + blk + static_cast<int64_t>(sizeof(bl::DecTail)) > static_cast<int64_t>(kDecMaxSmem))
-        continue;
+      const int64_t tail = static_cast<int64_t>(sizeof(bl::DecTail));
+      if (slots + blk + tail > static_cast<int64_t>(kDecMaxSmem)) continue;
+      // streaming: chunks of bpc blocks, `st` of them in flight
+      int64_t bpc = kDecStageTarget / blk;
+      if (bpc < 1) bpc = 1;
+      if (bpc > nblocks) bpc = nblocks;
+      const int64_t chunks = (nblocks + bpc - 1) / bpc;
+      int64_t ring = static_cast<int64_t>(kDecTwoCtaSmem) - slots - tail;
+      if (ring > kDecRingBytes) ring = kDecRingBytes;
+      if (ring < bpc * blk) ring = bpc * blk;
+      int64_t st = ring / (bpc * blk);
+      if (st > bl::kDecMaxStages) st = bl::kDecMaxStages;
+      if (st > chunks) st = chunks;
+      if (chunks > st) {
+        // A stage is refilled only after every warp has passed it, so the
+        // chunks go through one after another; a chunk takes as long as its
+        // busiest warp (a lone warp issues well below one instruction per
+        // cycle: 2.5 cycles per instruction) or the SM's issue slots.
+        const double t_chunk_warp = 2.5 * std::ceil(static_cast<double>(bpc) / teams) * per_block;
+        const double t_chunk_issue = static_cast<double>(bpc) * G * per_block / 4.0;
+        const double t_chunk = t_chunk_warp > t_chunk_issue ? t_chunk_warp : t_chunk_issue;
+        const double per_chunk_load = (kDecLoadLatency + t_chunk) / st;
+        const double t_stream =
+            kDecLoadLatency + chunks * (t_chunk > per_chunk_load ? t_chunk : per_chunk_load);
+        if (t_stream > cost) cost = t_stream;
+      }
       if (cost < best * 0.999) {
         best = cost;
         found = true;

@@ -55,7 +55,7 @@ namespace bl {
 constexpr int kDecComputeWarps = 16;
 constexpr int kDecComputeThreads = 32 * kDecComputeWarps;
 constexpr int kDecThreads = kDecComputeThreads + 32;  // + producer warp
-constexpr int kDecMaxStages = 4;
+constexpr int kDecMaxStages = 8;
 constexpr int kDecMaxBlocks = 64;  // row blocks per CTA when warps share a block (reduction slots)
 constexpr int kDecMaxMT = 4;
 
