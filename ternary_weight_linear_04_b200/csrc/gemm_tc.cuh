@@ -85,8 +85,9 @@ __global__ void __launch_bounds__(kTcThreads, BM <= 32 ? 2 : 1)
   using Cfg = TcCfg<BM>;
   constexpr int S = Cfg::kStages;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
+  // 1024-byte aligned base (the swizzle atom), by pointer arithmetic on the
+  // shared array so that every access below stays a shared-memory access
+  uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* sA = base;                    // [S] unpacked weights
   uint8_t* sB = sA + S * Cfg::kABytes;   // [S] activations
   uint8_t* sP = sB + S * Cfg::kBBytes;   // [S] packed weights

@@ -183,7 +183,10 @@ struct QVec<float> {
 
 // One 256-thread CTA per token row.  `vec` = the row can be read with
 // 16-byte loads (K a multiple of the vector width, x 16-byte aligned) and
-// xq written with 8/4-byte stores.
+// xq written with 8/4-byte stores.  The first kCache vectors of each thread
+// stay in registers between the absmax pass and the quantise pass (all of
+// the row for K up to 256 * 8 * kCache bf16 values), so the row is read
+// from memory once; longer rows read the rest again.
 template <typename T>
 __global__ void __launch_bounds__(256) k_quant_act(const T* __restrict__ x, int64_t M, int64_t K,
                                                     int vec, int8_t* __restrict__ xq,
@@ -192,6 +195,7 @@ __global__ void __launch_bounds__(256) k_quant_act(const T* __restrict__ x, int6
   __shared__ float redf[8];
   __shared__ int32_t redi[8];
   constexpr int V = QVec<T>::kN;
+  constexpr int kCache = 16 / V;  // 16 values per thread kept in registers
   constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -199,8 +203,18 @@ __global__ void __launch_bounds__(256) k_quant_act(const T* __restrict__ x, int6
     const T* row = x + m * K;
     int8_t* qrow = xq + m * K;
     float amax = 0.0f;
+    float cache[kCache][V];
     if (vec) {
-      for (int64_t k = static_cast<int64_t>(threadIdx.x) * V; k < K; k += 256 * V) {
+#pragma unroll
+      for (int c = 0; c < kCache; ++c) {
+        const int64_t k = (static_cast<int64_t>(threadIdx.x) + 256 * c) * V;
+        if (k < K) {
+          QVec<T>::load(row + k, cache[c]);
+#pragma unroll
+          for (int i = 0; i < V; ++i) amax = fmaxf(amax, fabsf(cache[c][i]));
+        }
+      }
+      for (int64_t k = (static_cast<int64_t>(threadIdx.x) + 256 * kCache) * V; k < K; k += 256 * V) {
         float f[V];
         QVec<T>::load(row + k, f);
 #pragma unroll
@@ -214,17 +228,25 @@ __global__ void __launch_bounds__(256) k_quant_act(const T* __restrict__ x, int6
     const float qs = quant_scale(eta);
     const bool eta_bf16 = is_bf16_value(eta);
     int32_t sum = 0;
+    auto quant_store = [&](int64_t k, const float (&f)[V]) {
+      int32_t q[V];
+#pragma unroll
+      for (int i = 0; i < V; ++i) {
+        q[i] = kBf16 ? quantise_bf16(f[i], eta, qs, eta_bf16) : quantise_fast(f[i], eta, qs);
+        sum += q[i];
+      }
+      QVec<T>::store(qrow + k, q);
+    };
     if (vec) {
-      for (int64_t k = static_cast<int64_t>(threadIdx.x) * V; k < K; k += 256 * V) {
+#pragma unroll
+      for (int c = 0; c < kCache; ++c) {
+        const int64_t k = (static_cast<int64_t>(threadIdx.x) + 256 * c) * V;
+        if (k < K) quant_store(k, cache[c]);
+      }
+      for (int64_t k = (static_cast<int64_t>(threadIdx.x) + 256 * kCache) * V; k < K; k += 256 * V) {
         float f[V];
         QVec<T>::load(row + k, f);
-        int32_t q[V];
-#pragma unroll
-        for (int i = 0; i < V; ++i) {
-          q[i] = kBf16 ? quantise_bf16(f[i], eta, qs, eta_bf16) : quantise_fast(f[i], eta, qs);
-          sum += q[i];
-        }
-        QVec<T>::store(qrow + k, q);
+        quant_store(k, f);
       }
     } else {
       for (int64_t k = threadIdx.x; k < K; k += 256) {
