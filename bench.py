@@ -629,7 +629,8 @@ def run_cpu_baseline(seconds):
 def run_reference(args, world, rank):
     """The CPU oracle timed on this machine's host cores: each step a bounded
     sample of the decode workload (a slice of output rows of both
-    matrices), sized so warm-up + steps take about two minutes."""
+    matrices), sized so warm-up + steps take about --ref-seconds (two
+    minutes by default)."""
     if rank != 0:
         return None
     from oracle import native as orc
@@ -654,7 +655,7 @@ def run_reference(args, world, rank):
     t0 = time.perf_counter()
     step(1.0)
     t_full = time.perf_counter() - t0
-    budget = 120.0 / max(1, args.steps + args.warmup)
+    budget = float(args.ref_seconds) / max(1, args.steps + args.warmup)
     frac = min(1.0, budget / max(t_full, 1e-9))
     for _ in range(args.warmup):
         step(frac)
@@ -689,6 +690,8 @@ def main():
                     help="comma list of extra sections: e2e,prefill,pack,sweep,layer70b,crossover")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--ref-seconds", type=float, default=120.0,
+                    help="--impl reference: total CPU time of warm-up + timed steps")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
