@@ -323,16 +323,19 @@ def _chk(status, what):
 
 
 def load_traffic(kernel):
-    """dram bytes per launch from the committed ncu summary, if present and
-    current (profiles/*.json written alongside the text summaries)."""
-    p = os.path.join(ROOT, "profiles", "traffic.json")
+    """DRAM bytes per launch of `kernel` from the committed ncu summary
+    (profiles/traffic.md, a markdown table), or None if absent."""
+    p = os.path.join(ROOT, "profiles", "traffic.md")
     if not os.path.exists(p):
         return None
-    try:
-        d = json.load(open(p))
-        return d.get(kernel)
-    except Exception:
-        return None
+    for line in open(p):
+        cells = [c.strip() for c in line.strip().strip("|").split("|")]
+        if len(cells) >= 2 and cells[0] == kernel:
+            try:
+                return int(cells[1])
+            except ValueError:
+                return None
+    return None
 
 
 def run_e2e(args, mats, M, stream, world):
@@ -410,6 +413,7 @@ def run_prefill(args, dev, stream, peaks, peak_src, world):
             "kernel": "k_gemm_tc", "us_per_forward": round(per * 1e6, 2),
             "tops": round(tops, 1), "int8_peak_tops": round(peak, 1),
             "frac": round(tops / peak, 4), "bound": "tensor",
+            "traffic": load_traffic("k_gemm_tc"),
             "peak_source": "%s bf16_tflops (burst) x %.0f nominal int8:bf16 ratio" % (peak_src, INT8_PER_BF16),
             "addsub_ops_needed_frac": "nnz(W~)/(N*K) of the dense ops (about 0.69)",
             "quant_us": round(tq * 1e6, 2), "quant_gbs": round(qbytes / tq / 1e9, 1)}
