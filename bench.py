@@ -419,10 +419,12 @@ def run_prefill(args, dev, stream, peaks, peak_src, world):
             "quant_us": round(tq * 1e6, 2), "quant_gbs": round(qbytes / tq / 1e9, 1)}
 
 
-def time_linear_step(mats, M, stream, world, min_seconds=0.25, xkey="x"):
+def time_linear_step(mats, M, stream, world, min_seconds=0.25, xkey="x", groups=None):
     """Seconds per step of one bitlinear_linear call per matrix (static
     weights), CUDA graph over every rotating packed copy, max over ranks.
-    mats: dicts with K, N, copies [(packed, gamma)], m[xkey] (>= M rows, bf16)."""
+    mats: dicts with K, N, copies [(packed, gamma)], m[xkey] (>= M rows, bf16).
+    groups: lists of matrix indices sharing one input, each run as one
+    bitlinear_linear_group call (the others one call each)."""
     from ternary_weight_linear_04_b200 import _lib
     L = _lib.lib()
     P = ctypes.c_void_p
@@ -443,8 +445,32 @@ def time_linear_step(mats, M, stream, world, min_seconds=0.25, xkey="x"):
              P(b["xsum"].data_ptr()), None, _lib.BL_FLAG_WEIGHTS_STATIC, sptr)
         return lambda: _chk(L.bitlinear_linear(*a), "linear")
 
+    def call_group(idx, c):
+        n = len(idx)
+        arr = ctypes.c_void_p * n
+        pk = arr(*[P(mats[i]["copies"][c][0].data_ptr()) for i in idx])
+        gm = arr(*[P(mats[i]["copies"][c][1].data_ptr()) for i in idx])
+        ns = (ctypes.c_int64 * n)(*[mats[i]["N"] for i in idx])
+        ys = arr(*[P(bufs[i]["y"].data_ptr()) for i in idx])
+        b0 = bufs[idx[0]]
+        a = (P(b0["x"].data_ptr()), _lib.BL_BF16, M, mats[idx[0]]["K"], n, pk, gm, ns, ys,
+             _lib.BL_BF16, _lib.BL_FLAG_WEIGHTS_STATIC, sptr)
+        keep = (pk, gm, ns, ys)
+        return lambda: (_chk(L.bitlinear_linear_group(*a), "linear_group"), keep)
+
     copies = len(mats[0]["copies"])
-    calls = [call(m, b, c) for c in range(copies) for m, b in zip(mats, bufs)]
+    if groups is None:
+        calls = [call(m, b, c) for c in range(copies) for m, b in zip(mats, bufs)]
+    else:
+        grouped = {i for g in groups for i in g}
+        calls = []
+        for c in range(copies):
+            for i, (m, b) in enumerate(zip(mats, bufs)):
+                g = next((g for g in groups if g[0] == i), None)
+                if g is not None:
+                    calls.append(call_group(g, c))
+                elif i not in grouped:
+                    calls.append(call(m, b, c))
     with torch.cuda.stream(stream):
         for fn in calls:
             fn()
@@ -512,7 +538,13 @@ def run_layer70b(dev, stream, world, peaks, l2):
         t = time_linear_step(mats, M, stream, world)
         b = sum(linear_bytes(M, m["K"], m["N"]) for m in mats)
         rows.append({"M": M, "us_per_layer": round(t * 1e6, 2), "gbs": round(b / t / 1e9, 1),
-                     "frac": round(b / t / 1e9 / hbm, 4)})
+                     "frac": round(b / t / 1e9 / hbm, 4), "launches": 7 if M <= 4 else 14})
+    # shared-input fusion: Wq|Wk|Wv and gate|up each as one grouped launch
+    t = time_linear_step(mats, 1, stream, world, groups=[[0, 1, 2], [4, 5]])
+    b = sum(linear_bytes(1, m["K"], m["N"]) for m in mats)
+    rows.append({"M": 1, "grouped": "Wq|Wk|Wv and gate|up (bitlinear_linear_group)",
+                 "us_per_layer": round(t * 1e6, 2), "gbs": round(b / t / 1e9, 1),
+                 "frac": round(b / t / 1e9 / hbm, 4), "launches": 4})
     del mats
     torch.cuda.empty_cache()
     return {"workload": "layer_70b: Wq 8192^2, Wk/Wv 8192x1024, Wo 8192^2, gate/up 8192x28672, "

@@ -269,6 +269,39 @@ bl_status bitlinear_set_decode_shape(int team_warps, int rows_per_block);
  */
 bl_status bitlinear_set_tc_split(int k_split);
 
+/*
+ * bitlinear_linear for up to 4 matrices that share one activation input
+ * (a decoder layer's Wq|Wk|Wv, or gate|up) in ONE launch of the fused decode
+ * kernel: every CTA quantises x itself and works on rows of one matrix,
+ * each with its own gamma and output.  The page "BitNet b1.58 & 1-Bit LLM
+ * Architectures: Eliminating Matrix Multiplication and Running 70B Models on
+ * CPU in 2026", section 2, names the seven BitLinear projections of a
+ * Transformer block (Wq, Wk, Wv, Wo and Wgate, Wup, Wdown), of which Wq|Wk|Wv
+ * and Wgate|Wup read the same input; it gives no fused form.  The results are
+ * those of bitlinear_linear on each matrix, bit for bit.
+ *
+ *   x         in   bf16 M x K row-major, 16-byte aligned (xdt must be
+ *                  BL_BF16; BL_ERR_UNSUPPORTED otherwise).
+ *   M, K      in   1 <= M <= 4, K % 64 == 0, K * M' <= 131072 (the fused
+ *                  decode kernel's range; BL_ERR_UNSUPPORTED otherwise).
+ *                  M = 0 is a no-op.
+ *   nseg      in   1..4 matrices.
+ *   packed[s], gamma[s], N[s]   in   host arrays of nseg device pointers /
+ *                  row counts: matrix s as bitlinear_pack_weights wrote it
+ *                  (N[s] x ceil(K/4), 16-byte aligned) and its gamma.
+ *   y[s]      out  host array of nseg device pointers: M x N[s] row-major,
+ *                  fp32 or bf16 (ydt), 16-byte aligned.
+ *   flags     in   0 or BL_FLAG_WEIGHTS_STATIC (for every matrix).
+ * x~, eta, xsum and y_int are not returned (use bitlinear_linear).
+ * Errors: BL_ERR_INVALID_ARG for nseg outside 1..4, null pointers or
+ * arrays, N[s] < 1, unknown dtypes; BL_ERR_UNSUPPORTED as above;
+ * BL_ERR_ALIGNMENT for misaligned pointers.
+ */
+bl_status bitlinear_linear_group(const void* x, bl_dtype xdt, int64_t M, int64_t K, int nseg,
+                                 const uint8_t* const* packed, const float* const* gamma,
+                                 const int64_t* N, void* const* y, bl_dtype ydt, unsigned flags,
+                                 void* stream);
+
 /* The path bitlinear_forward would pick for these sizes and pointers. */
 bl_path bitlinear_select_path(int64_t M, int64_t K, int64_t N,
                               const void* xq, const void* packed, const void* y,

@@ -160,6 +160,31 @@ def linear(x, packed, gamma, N, out_dtype=torch.bfloat16, want_quant=False, want
     return out_[0] if len(out_) == 1 else out_
 
 
+def linear_group(x, packed, gamma, out_dtype=torch.bfloat16, weights_static=False, stream=None,
+                 out=None):
+    """bitlinear_linear_group: the per-token layer for up to 4 matrices that
+    share the activations x (bf16 M x K, M <= 4), in one launch.  packed and
+    gamma are lists (one per matrix); returns the list of outputs."""
+    _require_cuda(x, *packed, *gamma)
+    if x.dim() != 2 or x.dtype != torch.bfloat16:
+        raise ValueError("x must be a 2-D bfloat16 tensor")
+    M, K = x.shape
+    n = len(packed)
+    if n != len(gamma) or not 1 <= n <= 4:
+        raise ValueError("one gamma per packed matrix, 1 to 4 matrices")
+    Ns = [p.shape[0] for p in packed]
+    for p in packed:
+        if p.shape[1] != (K + 3) // 4:
+            raise ValueError("packed shape %s does not match K=%d" % (tuple(p.shape), K))
+    ys = out if out is not None else [torch.empty((M, N), dtype=out_dtype, device=x.device) for N in Ns]
+    arr = ctypes.c_void_p * n
+    check(_lib.lib().bitlinear_linear_group(
+        _ptr(x), _lib.BL_BF16, M, K, n, arr(*[_ptr(p) for p in packed]), arr(*[_ptr(g) for g in gamma]),
+        (ctypes.c_int64 * n)(*Ns), arr(*[_ptr(y) for y in ys]), _DTYPES[ys[0].dtype],
+        _lib.BL_FLAG_WEIGHTS_STATIC if weights_static else 0, _stream(stream)), "bitlinear_linear_group")
+    return ys
+
+
 def select_path(M, K, N, xq, packed, y, y_int=None):
     return PATH_NAMES[int(_lib.lib().bitlinear_select_path(M, K, N, _ptr(xq), _ptr(packed),
                                                            _ptr(y), _ptr(y_int)))]

@@ -334,8 +334,24 @@ template <int MT, typename XT, typename OutT>
 bl_status launch_decode_kernel(const bl::DecodeArgs& a0, int sms, cudaStream_t st) {
   constexpr int64_t kXElem = std::is_same<XT, bl::DecNoFuse>::value ? 1 : 2;
   DecGeom g;
-  if (!decode_geometry(MT, a0.M, a0.K, a0.N, sms, kXElem, &g)) return BL_ERR_UNSUPPORTED;
+  // a group of matrices sharing the activations: shape from the summed rows
+  int64_t n_total = a0.N;
+  if (a0.nseg > 0) {
+    n_total = 0;
+    for (int s = 0; s < a0.nseg; ++s) n_total += a0.seg_N[s];
+  }
+  if (!decode_geometry(MT, a0.M, a0.K, n_total, sms, kXElem, &g)) return BL_ERR_UNSUPPORTED;
   bl::DecodeArgs a = a0;
+  if (a0.nseg > 0) {  // whole CTAs per matrix, the same rows per CTA for all of them
+    int64_t cta = 0;
+    for (int s = 0; s < a0.nseg; ++s) {
+      a.seg_cta0[s] = static_cast<int>(cta);
+      cta += (a0.seg_N[s] + g.rows_per_cta - 1) / g.rows_per_cta;
+    }
+    a.seg_cta0[a0.nseg] = static_cast<int>(cta);
+    if (cta > 0x7FFFFFFF) return BL_ERR_UNSUPPORTED;
+    g.grid = static_cast<int>(cta);
+  }
   a.rows_per_cta = g.rows_per_cta;
   a.blocks_per_chunk = g.bpc;
   a.stages = g.stages;
@@ -517,6 +533,45 @@ const char* bitlinear_status_str(bl_status status) {
     case BL_ERR_TIMEOUT: return "a kernel gave up a bounded wait";
   }
   return "unknown status";
+}
+
+bl_status bitlinear_linear_group(const void* x, bl_dtype xdt, int64_t M, int64_t K, int nseg,
+                                 const uint8_t* const* packed, const float* const* gamma,
+                                 const int64_t* N, void* const* y, bl_dtype ydt, unsigned flags,
+                                 void* stream) {
+  if (nseg < 1 || nseg > bl::kDecMaxSeg || !packed || !gamma || !N || !y) return BL_ERR_INVALID_ARG;
+  if (M < 0 || K < 1) return BL_ERR_INVALID_ARG;
+  if ((xdt != BL_F32 && xdt != BL_BF16) || (ydt != BL_F32 && ydt != BL_BF16))
+    return BL_ERR_INVALID_ARG;
+  for (int s = 0; s < nseg; ++s) {
+    if (!packed[s] || !gamma[s] || N[s] < 1) return BL_ERR_INVALID_ARG;
+    if (M > 0 && !y[s]) return BL_ERR_INVALID_ARG;
+  }
+  if (M == 0) return BL_OK;
+  if (!x) return BL_ERR_INVALID_ARG;
+  if (xdt != BL_BF16 || !decode_ok(M, K)) return BL_ERR_UNSUPPORTED;
+  if (!aligned(x, 16)) return BL_ERR_ALIGNMENT;
+  for (int s = 0; s < nseg; ++s) {
+    if (N[s] > INT32_MAX / 2) return BL_ERR_UNSUPPORTED;
+    if (!aligned(packed[s], 16) || !aligned(y[s], 16) || !aligned(gamma[s], 4)) return BL_ERR_ALIGNMENT;
+  }
+  int sms = 148;
+  bl_status st = device_info(&sms);
+  if (st != BL_OK) return st;
+  bl::DecodeArgs a = {};
+  a.x = x; a.M = static_cast<int>(M); a.K = static_cast<int>(K);
+  a.N = static_cast<int>(N[0]); a.packed = packed[0]; a.gamma = gamma[0]; a.y = y[0];
+  a.weights_static = (flags & BL_FLAG_WEIGHTS_STATIC) ? 1 : 0;
+  a.nseg = nseg;
+  for (int s = 0; s < nseg; ++s) {
+    a.seg_packed[s] = packed[s];
+    a.seg_gamma[s] = gamma[s];
+    a.seg_y[s] = y[s];
+    a.seg_N[s] = static_cast<int>(N[s]);
+  }
+  const cudaStream_t cs = as_stream(stream);
+  return ydt == BL_F32 ? launch_decode<__nv_bfloat16, float>(a, sms, cs)
+                       : launch_decode<__nv_bfloat16, __nv_bfloat16>(a, sms, cs);
 }
 
 bl_status bitlinear_decode_shape(int64_t M, int64_t K, int64_t N, int fused, int32_t* shape) {

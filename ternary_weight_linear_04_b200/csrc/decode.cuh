@@ -58,6 +58,7 @@ constexpr int kDecThreads = kDecComputeThreads + 32;  // + producer warp
 constexpr int kDecMaxStages = 8;
 constexpr int kDecMaxBlocks = 64;  // row blocks per CTA when warps share a block (reduction slots)
 constexpr int kDecMaxMT = 4;
+constexpr int kDecMaxSeg = 4;  // matrices sharing one activation input in one launch
 
 __device__ __forceinline__ void bulk_load_1d(void* smem_dst, const void* gsrc, uint32_t bytes,
                                              uint64_t* bar) {
@@ -107,6 +108,15 @@ struct DecodeArgs {
   int8_t* xq_out;        // fused, optional: CTA 0 writes x~, eta, xsum
   float* eta_out;
   int32_t* xsum_out;
+  // Several matrices sharing these activations (nseg >= 1): CTAs
+  // [seg_cta0[s], seg_cta0[s+1]) work on segment s, whose packed weights,
+  // gamma, output and row count replace packed / gamma / y / N above.
+  int nseg;              // 0 = the single matrix above
+  int seg_cta0[kDecMaxSeg + 1];
+  const uint8_t* seg_packed[kDecMaxSeg];
+  const float* seg_gamma[kDecMaxSeg];
+  void* seg_y[kDecMaxSeg];
+  int seg_N[kDecMaxSeg];
 };
 
 // Shared memory after the stages: barriers, flags, per-token values and the
@@ -193,8 +203,18 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode(const DecodeArgs a) {
   DecTail& T = *reinterpret_cast<DecTail*>(stages + S * stage_bytes);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int r_begin = blockIdx.x * a.rows_per_cta;
-  const int nrows = max(0, min(a.N - r_begin, a.rows_per_cta));
+  // this CTA's matrix (one of several sharing the activations, or the only one)
+  int cta = blockIdx.x, seg = 0;
+  if (a.nseg > 0) {
+    while (seg + 1 < a.nseg && cta >= a.seg_cta0[seg + 1]) ++seg;
+    cta -= a.seg_cta0[seg];
+  }
+  const uint8_t* const packed = a.nseg > 0 ? a.seg_packed[seg] : a.packed;
+  const float* const gamma_p = a.nseg > 0 ? a.seg_gamma[seg] : a.gamma;
+  void* const y_out = a.nseg > 0 ? a.seg_y[seg] : a.y;
+  const int N = a.nseg > 0 ? a.seg_N[seg] : a.N;
+  const int r_begin = cta * a.rows_per_cta;
+  const int nrows = max(0, min(N - r_begin, a.rows_per_cta));
   const int nblocks = (nrows + RB - 1) / RB;
   const int nchunks = (nrows + rows_per_chunk - 1) / rows_per_chunk;
   const int acc_warps = a.teams * G;
@@ -207,7 +227,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode(const DecodeArgs a) {
       const uint32_t bytes = static_cast<uint32_t>(rows) * static_cast<uint32_t>(P);
       mbar_arrive_expect_tx(&T.full[s], bytes);
       bulk_load_1d(stages + s * stage_bytes,
-                   a.packed + static_cast<int64_t>(r_begin + c * rows_per_chunk) * P, bytes,
+                   packed + static_cast<int64_t>(r_begin + c * rows_per_chunk) * P, bytes,
                    &T.full[s]);
     };
     const int first = min(S, nchunks);
@@ -221,7 +241,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode(const DecodeArgs a) {
       mbar_init_fence();
       if (a.weights_static) {
         for (int c = 0; c < first; ++c) issue(c);
-        T.gamma = *a.gamma;
+        T.gamma = *gamma_p;
       }
       pdl_wait();  // the preceding grid is complete and its writes are visible
       // Only now let the next grid launch: every SM then holds exactly this
@@ -236,7 +256,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode(const DecodeArgs a) {
       }
       if (!a.weights_static) {
         for (int c = 0; c < first; ++c) issue(c);
-        T.gamma = *a.gamma;
+        T.gamma = *gamma_p;
       }
     }
     __syncwarp();
@@ -433,8 +453,8 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode(const DecodeArgs a) {
         const int r = v / MT, m = v - r * MT;
         if (r < brows && m < a.M) {
           const int32_t yi = total - T.s_xsum[m];
-          const int64_t o = static_cast<int64_t>(m) * a.N + r_begin + row0 + r;
-          store_out<OutT>(a.y, o, rescale(yi, T.s_scale[m]));
+          const int64_t o = static_cast<int64_t>(m) * N + r_begin + row0 + r;
+          store_out<OutT>(y_out, o, rescale(yi, T.s_scale[m]));
           if (a.y_int) a.y_int[o] = yi;
           if constexpr (kFused) {
             if (blockIdx.x == 0 && b == 0 && r == 0 && a.xsum_out) a.xsum_out[m] = T.s_xsum[m];

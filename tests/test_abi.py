@@ -94,6 +94,18 @@ def test_bad_arguments_are_rejected_without_a_launch(L):
     assert L.bitlinear_set_tc_split(-1) == _lib.BL_ERR_INVALID_ARG
     assert L.bitlinear_set_tc_split(9) == _lib.BL_ERR_INVALID_ARG
     assert L.bitlinear_set_tc_split(0) == _lib.BL_OK
+    grp = L.bitlinear_linear_group
+    arr1 = (ctypes.c_void_p * 1)(fake)
+    n1 = (ctypes.c_int64 * 1)(64)
+    assert grp(fake, 1, 1, 64, 0, arr1, arr1, n1, arr1, 1, 0, None) == _lib.BL_ERR_INVALID_ARG  # nseg 0
+    assert grp(fake, 1, 1, 64, 5, arr1, arr1, n1, arr1, 1, 0, None) == _lib.BL_ERR_INVALID_ARG  # nseg 5
+    assert grp(fake, 1, 1, 64, 1, None, arr1, n1, arr1, 1, 0, None) == _lib.BL_ERR_INVALID_ARG
+    assert grp(fake, 1, 1, 64, 1, arr1, arr1, (ctypes.c_int64 * 1)(0), arr1, 1, 0, None) == _lib.BL_ERR_INVALID_ARG
+    assert grp(fake, 0, 1, 64, 1, arr1, arr1, n1, arr1, 1, 0, None) == _lib.BL_ERR_UNSUPPORTED  # f32 x
+    assert grp(fake, 1, 5, 64, 1, arr1, arr1, n1, arr1, 1, 0, None) == _lib.BL_ERR_UNSUPPORTED  # M > 4
+    assert grp(fake, 1, 1, 96, 1, arr1, arr1, n1, arr1, 1, 0, None) == _lib.BL_ERR_UNSUPPORTED  # K % 64
+    assert grp(P(257), 1, 1, 64, 1, arr1, arr1, n1, arr1, 1, 0, None) == _lib.BL_ERR_ALIGNMENT
+    assert grp(None, 1, 0, 64, 1, arr1, arr1, n1, arr1, 1, 0, None) == _lib.BL_OK  # M = 0
 
 
 def test_path_selection_is_host_logic(L):

@@ -508,3 +508,34 @@ def test_quantiser_tiny_rows_use_the_eta_floor():
                                       out_dtype=torch.float32, want_quant=True)
     np.testing.assert_array_equal(xq2.cpu().numpy(), ref_xq)
     np.testing.assert_array_equal(xsum2.cpu().numpy(), ref_xsum)
+
+
+# ----------------------------------------------------------------- shared-input groups
+
+@pytest.mark.parametrize("M", [1, 2, 3, 4])
+@pytest.mark.parametrize("Ns", [(1000, 256, 256), (3000, 3000), (777,), (130, 2, 517, 64)])
+def test_linear_group_matches_each_matrix(M, Ns):
+    """Up to 4 matrices sharing x in one launch: each output equals the
+    oracle's layer on its own matrix (and bitlinear_linear on it)."""
+    K = 4096
+    packs, gams, refs = [], [], []
+    x = None
+    for i, N in enumerate(Ns):
+        W, xi = inputs.make_case(8100 + 13 * i + N + M, M, K, N, act_dtype="bf16")
+        if x is None:
+            x = xi
+        ref_packed, ref_gamma, _ = orc.pack_weights(W)
+        _, _, packed, gamma = gpu_pack(W)
+        packs.append(packed); gams.append(gamma)
+        ref_xq, ref_eta, _ = orc.quant_act(x)
+        refs.append(orc.forward(ref_xq, ref_eta, ref_packed, ref_gamma, K, N)[1])
+    xd = torch.from_numpy(x).cuda().to(torch.bfloat16)
+    for static in (False, True):
+        ys = bl.linear_group(xd, packs, gams, out_dtype=torch.bfloat16, weights_static=static)
+        for y, ref_y, p, g in zip(ys, refs, packs, gams):
+            np.testing.assert_array_equal(y_bits(y.cpu()), orc.f32_to_bf16_bits(ref_y))
+            y1 = bl.linear(xd, p, g, p.shape[0], out_dtype=torch.bfloat16, weights_static=static)
+            np.testing.assert_array_equal(y_bits(y1.cpu()), y_bits(y.cpu()))
+    ys = bl.linear_group(xd, packs, gams, out_dtype=torch.float32)
+    for y, ref_y in zip(ys, refs):
+        np.testing.assert_array_equal(y.cpu().numpy().view(np.uint32), ref_y.view(np.uint32))
