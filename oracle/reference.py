@@ -17,6 +17,10 @@ Citations (page title tags as in ``bitlinear_oracle.c``):
   2-bit codes and bit order -- [Production] "Production Deployment Standards"
                                guideline 1; [No-Multiply] "Kernel
                                Implementation: The Lookup Table Approach"
+  base-3 packing            -- [Additive] "Energy, Memory Bandwidth, and
+                               Serving Economics" (compact ternary packing,
+                               named only: the layout is this build's
+                               reading, see pack3)
   rescale                   -- [Production] pipeline figure step 5,
                                BitLinear158.forward
 """
@@ -80,6 +84,50 @@ def unpack2(packed, K):
     if np.any(codes == 3):
         raise ValueError("invalid 2-bit code 11 in packed weights")
     return (codes[:, :K].astype(np.int8) - 1)
+
+
+def packed3_stride(K):
+    """Row stride of the base-3 layout: ceil(K/5) bytes rounded up to a
+    multiple of 16 (this build's reading; the pages give no layout)."""
+    return 16 * ((((K + 4) // 5) + 15) // 16)
+
+
+POW3 = np.array([1, 3, 9, 27, 81], dtype=np.int64)
+
+
+def pack3(t):
+    """Base-3 "compact ternary packing" ([Additive] "Energy, Memory Bandwidth,
+    and Serving Economics"; 3^5 = 243 <= 256): byte g of a row holds the trits
+    5g .. 5g+4 as sum_j (t + 1) * 3^j.  Trits past K are 0; the row is padded
+    to packed3_stride(K) with bytes of five zero trits (value 121).
+    Returns N x packed3_stride(K) uint8."""
+    t = np.asarray(t, dtype=np.int8)
+    N, K = t.shape
+    S = packed3_stride(K)
+    digits = np.ones((N, 5 * S), dtype=np.int64)   # digit = t + 1; padding digit 1 (t = 0)
+    digits[:, :K] = t.astype(np.int64) + 1
+    return (digits.reshape(N, S, 5) * POW3).sum(axis=2).astype(np.uint8)
+
+
+def unpack3(packed3, K):
+    """Inverse of pack3: the base-3 digits of each byte, least significant
+    first, minus one; byte values above 242 are rejected."""
+    b = np.asarray(packed3, dtype=np.uint8).astype(np.int64)
+    N, S = b.shape
+    if S != packed3_stride(K):
+        raise ValueError("packed3 width does not match K")
+    if np.any(b > 242):
+        raise ValueError("byte above 242 in base-3 packed weights")
+    digits = np.stack([(b // int(p)) % 3 for p in POW3], axis=2).reshape(N, 5 * S)
+    return (digits[:, :K] - 1).astype(np.int8)
+
+
+def forward3(xq, eta, packed3, gamma, K):
+    """The layer on base-3 packed weights: the same trits, so the same
+    (y_int, y) as forward() on the 2-bit packing of them."""
+    t = unpack3(packed3, K)
+    y_int = accumulate(xq, t)
+    return y_int, rescale(y_int, eta, gamma)
 
 
 def pack_weights(W):
