@@ -293,7 +293,7 @@ def run_ours(args, world, rank, local):
            "clocks": clk.summary()}
 
     sections = (set(args.sections.split(",")) if args.sections else
-                {"e2e", "prefill", "pack", "sweep", "layer70b", "crossover"})
+                {"e2e", "prefill", "pack", "sweep", "layer70b", "crossover", "base3"})
     if args.quick:
         sections = set()
     if "e2e" in sections:
@@ -312,6 +312,8 @@ def run_ours(args, world, rank, local):
         out["layer_70b"] = run_layer70b(dev, stream, world, peaks, l2)
     if "crossover" in sections:
         out["crossover"] = run_crossover(dev, stream, world, peaks, l2)
+    if "base3" in sections:
+        out["base3"] = run_base3(dev, stream, world, peaks, l2)
     if (rank == 0) and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = run_cpu_baseline(args.cpu_seconds)
     return out
@@ -608,6 +610,76 @@ def run_crossover(dev, stream, world, peaks, l2):
                                                            "takes M <= 4 and is faster there)"}
 
 
+def run_base3(dev, stream, world, peaks, l2):
+    """Base-3 packing (five trits per byte) against the 2-bit codes, x~ given,
+    M = 1: the accumulate kernels on decode_3b and on 8192x28672."""
+    from ternary_weight_linear_04_b200 import _lib, inputs
+    from ternary_weight_linear_04_b200 import bitlinear as bl
+    L = _lib.lib()
+    P = ctypes.c_void_p
+    sptr = ctypes.c_void_p(stream.cuda_stream)
+    hbm = float(peaks["hbm_gbs"])
+    rows = []
+    for wl_name in ("decode_3b", "outlier_sweep"):
+        wl = inputs.WORKLOADS[wl_name]
+        mats = []
+        for j, mat in enumerate(wl.matrices):
+            W, x = inputs.make_matrix_inputs(wl, j, m_max=1)
+            with torch.cuda.stream(stream):
+                Wd = torch.from_numpy(W).to(dev)
+                p2, g = bl.pack_weights(Wd, stream=stream)
+                p3, _ = bl.pack_weights3(Wd, stream=stream)
+                xq, eta, xsum = bl.quant_act(torch.from_numpy(x).to(dev).to(torch.bfloat16), stream=stream)
+            torch.cuda.synchronize()
+            del Wd, W
+            mats.append(dict(K=mat.K, N=mat.N, p2=p2, p3=p3, g=g, xq=xq, eta=eta, xsum=xsum,
+                             y=torch.empty((1, mat.N), dtype=torch.bfloat16, device=dev)))
+        b2 = sum(m["N"] * ((m["K"] + 3) // 4) for m in mats)
+        b3 = sum(m["p3"].numel() for m in mats)
+        copies = max(2, int(np.ceil(3 * l2 / b3)))
+        for m in mats:
+            m["c2"] = [m["p2"]] + [m["p2"].clone() for _ in range(copies - 1)]
+            m["c3"] = [m["p3"]] + [m["p3"].clone() for _ in range(copies - 1)]
+        torch.cuda.synchronize()
+        res = {"workload": wl_name, "packed_bytes_2bit": b2, "packed_bytes_base3": b3}
+        for fmt in ("2bit", "base3"):
+            calls = []
+            for c in range(copies):
+                for m in mats:
+                    if fmt == "2bit":
+                        a = (P(m["xq"].data_ptr()), P(m["eta"].data_ptr()), P(m["xsum"].data_ptr()), 1,
+                             m["K"], P(m["c2"][c].data_ptr()), P(m["g"].data_ptr()), m["N"],
+                             P(m["y"].data_ptr()), _lib.BL_BF16, None, _lib.BL_PATH_GEMV,
+                             _lib.BL_FLAG_WEIGHTS_STATIC, sptr)
+                        calls.append(lambda a=a: _chk(L.bitlinear_forward_path(*a), "forward"))
+                    else:
+                        a = (P(m["xq"].data_ptr()), P(m["eta"].data_ptr()), P(m["xsum"].data_ptr()), 1,
+                             m["K"], P(m["c3"][c].data_ptr()), P(m["g"].data_ptr()), m["N"],
+                             P(m["y"].data_ptr()), _lib.BL_BF16, None, sptr)
+                        calls.append(lambda a=a: _chk(L.bitlinear_forward3(*a), "forward3"))
+            with torch.cuda.stream(stream):
+                for fn in calls:
+                    fn()
+            torch.cuda.synchronize()
+            gr = Capture(calls, stream)
+            with torch.cuda.stream(stream):
+                gr.replay()
+            torch.cuda.synchronize()
+            reps = 20
+            t = max_over_ranks(timed(lambda: [gr.replay() for _ in range(reps)], stream, world),
+                               world) / (reps * copies)
+            wb = b2 if fmt == "2bit" else b3
+            res[fmt] = {"us_per_step": round(t * 1e6, 2), "weight_gbs": round(wb / t / 1e9, 1),
+                        "hbm_frac": round(wb / t / 1e9 / hbm, 4),
+                        "trits_per_ns": round(sum(m["N"] * m["K"] for m in mats) / t / 1e9, 1)}
+        rows.append(res)
+        del mats
+        torch.cuda.empty_cache()
+    return {"what": "accumulate kernels only (x~ given), M=1: bitlinear_forward (2-bit codes, "
+                    "decode kernel) against bitlinear_forward3 (base-3, five trits per byte)",
+            "rows": rows}
+
+
 def run_pack(mats, stream, world):
     from ternary_weight_linear_04_b200 import bitlinear as bl
     m = mats[0]
@@ -723,7 +795,7 @@ def main():
     ap.add_argument("--m", type=int, default=1, help="tokens per step (decode batch)")
     ap.add_argument("--quick", action="store_true", help="headline only (no e2e/prefill/pack)")
     ap.add_argument("--sections", default="",
-                    help="comma list of extra sections: e2e,prefill,pack,sweep,layer70b,crossover")
+                    help="comma list of extra sections: e2e,prefill,pack,sweep,layer70b,crossover,base3")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-seconds", type=float, default=120.0,

@@ -302,6 +302,45 @@ bl_status bitlinear_linear_group(const void* x, bl_dtype xdt, int64_t M, int64_t
                                  const int64_t* N, void* const* y, bl_dtype ydt, unsigned flags,
                                  void* stream);
 
+/*
+ * Base-3 "compact ternary packing" (five trits per byte, 1.6 bits per
+ * weight): the measured alternative to the 2-bit codes.  The page "1-Bit
+ * Large Language Models and BitNet b1.58: How Ternary Weights and Additive
+ * Kernels Eliminate Matrix Multiplications", section "Energy, Memory
+ * Bandwidth, and Serving Economics", names the packing but gives no layout;
+ * this library's layout: byte g of row n holds the trits of columns
+ * 5g .. 5g+4 as sum_j (t + 1) * 3^j (least significant first), trits past K
+ * are 0, and a row is bitlinear_packed3_stride(K) = 16 * ceil(ceil(K/5)/16)
+ * bytes (padding bytes hold five zero trits, value 121).
+ */
+
+/* Row stride of the base-3 layout in bytes (0 if K < 1). */
+int64_t bitlinear_packed3_stride(int64_t K);
+
+/*
+ * bitlinear_pack_weights into the base-3 layout: the same gamma and the same
+ * trits, packed3 = N x bitlinear_packed3_stride(K) uint8.  Same arguments,
+ * workspace and errors as bitlinear_pack_weights.
+ */
+bl_status bitlinear_pack_weights3(const float* W, int64_t N, int64_t K, uint8_t* packed3,
+                                  float* gamma, void* workspace, void* stream);
+
+/*
+ * bitlinear_forward on base-3 packed weights (x~ given): the same y and
+ * y_int, bit for bit, as bitlinear_forward on the 2-bit packing of the same
+ * trits.  One CUDA-core kernel per 4 tokens or fewer (meant for decode
+ * batches; fewer per launch for long rows).
+ *   packed3   in   N x bitlinear_packed3_stride(K) uint8, 16-byte aligned.
+ *   other arguments as bitlinear_forward (y_int optional).
+ * Errors: BL_ERR_INVALID_ARG for null pointers, M < 0, K or N < 1 or an
+ * unknown ydt; BL_ERR_UNSUPPORTED when K is too large for the activation
+ * slots in shared memory (K above 29360) or N > 2^30;
+ * BL_ERR_ALIGNMENT for misaligned pointers.  M = 0 is a no-op.
+ */
+bl_status bitlinear_forward3(const int8_t* xq, const float* eta, const int32_t* xsum, int64_t M,
+                             int64_t K, const uint8_t* packed3, const float* gamma, int64_t N,
+                             void* y, bl_dtype ydt, int32_t* y_int, void* stream);
+
 /* The path bitlinear_forward would pick for these sizes and pointers. */
 bl_path bitlinear_select_path(int64_t M, int64_t K, int64_t N,
                               const void* xq, const void* packed, const void* y,

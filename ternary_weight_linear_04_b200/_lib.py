@@ -38,6 +38,9 @@ SIGNATURES = {
     "bitlinear_set_decode_shape": (_I, [_I, _I]),
     "bitlinear_set_tc_split": (_I, [_I]),
     "bitlinear_linear_group": (_I, [_P, _I, _I64, _I64, _I, _P, _P, _P, _P, _I, ctypes.c_uint, _P]),
+    "bitlinear_packed3_stride": (_I64, [_I64]),
+    "bitlinear_pack_weights3": (_I, [_P, _I64, _I64, _P, _P, _P, _P]),
+    "bitlinear_forward3": (_I, [_P, _P, _P, _I64, _I64, _P, _P, _I64, _P, _I, _P, _P]),
 }
 
 _lib = None

@@ -185,6 +185,40 @@ def linear_group(x, packed, gamma, out_dtype=torch.bfloat16, weights_static=Fals
     return ys
 
 
+def packed3_stride(K):
+    """Row stride (bytes) of the base-3 layout."""
+    return int(_lib.lib().bitlinear_packed3_stride(K))
+
+
+def pack_weights3(W, stream=None, workspace=None):
+    """bitlinear_pack_weights3: (packed3 N x stride uint8, gamma) on W's device."""
+    _require_cuda(W)
+    N, K = W.shape
+    dev = W.device
+    packed3 = torch.empty((N, packed3_stride(K)), dtype=torch.uint8, device=dev)
+    gamma = torch.empty(1, dtype=torch.float32, device=dev)
+    ws = workspace if workspace is not None else torch.empty(
+        int(_lib.lib().bitlinear_pack_workspace_bytes()), dtype=torch.uint8, device=dev)
+    check(_lib.lib().bitlinear_pack_weights3(_ptr(W), N, K, _ptr(packed3), _ptr(gamma), _ptr(ws),
+                                             _stream(stream)), "bitlinear_pack_weights3")
+    return packed3, gamma
+
+
+def forward3(xq, eta, xsum, packed3, gamma, N, out_dtype=torch.float32, want_int=False,
+             stream=None, out=None):
+    """bitlinear_forward3: the accumulate + rescale on base-3 packed weights."""
+    _require_cuda(xq, eta, xsum, packed3, gamma)
+    M, K = xq.shape
+    if packed3.shape != (N, packed3_stride(K)):
+        raise ValueError("packed3 shape %s does not match N=%d, K=%d" % (tuple(packed3.shape), N, K))
+    y = out if out is not None else torch.empty((M, N), dtype=out_dtype, device=xq.device)
+    y_int = torch.empty((M, N), dtype=torch.int32, device=xq.device) if want_int else None
+    check(_lib.lib().bitlinear_forward3(_ptr(xq), _ptr(eta), _ptr(xsum), M, K, _ptr(packed3), _ptr(gamma),
+                                        N, _ptr(y), _DTYPES[y.dtype], _ptr(y_int), _stream(stream)),
+          "bitlinear_forward3")
+    return (y, y_int) if want_int else y
+
+
 def select_path(M, K, N, xq, packed, y, y_int=None):
     return PATH_NAMES[int(_lib.lib().bitlinear_select_path(M, K, N, _ptr(xq), _ptr(packed),
                                                            _ptr(y), _ptr(y_int)))]

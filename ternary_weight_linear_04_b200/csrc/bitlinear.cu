@@ -18,6 +18,7 @@
 #include "bitlinear.h"
 #include "common.cuh"
 #include "decode.cuh"
+#include "base3.cuh"
 #include "gemm_tc.cuh"
 #include "gemv.cuh"
 #include "pack.cuh"
@@ -139,11 +140,15 @@ bool ensure_smem(Kern kern, size_t bytes, int* done_flags) {
   if (done_flags[dev] >= static_cast<int>(bytes) && done_flags[dev] > 0) return true;
   if (bytes > 48 * 1024 &&
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(bytes)) != cudaSuccess)
+                           static_cast<int>(bytes)) != cudaSuccess) {
+    (void)cudaGetLastError();  // do not leave the error for the next launch check
     return false;
+  }
   if (cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
-                           cudaSharedmemCarveoutMaxShared) != cudaSuccess)
+                           cudaSharedmemCarveoutMaxShared) != cudaSuccess) {
+    (void)cudaGetLastError();
     return false;
+  }
   done_flags[dev] = bytes > 0 ? static_cast<int>(bytes) : 1;
   return true;
 }
@@ -645,6 +650,87 @@ bl_status bitlinear_pack_weights(const float* W, int64_t N, int64_t K, uint8_t* 
   if (pctas > static_cast<int64_t>(sms) * 32) pctas = static_cast<int64_t>(sms) * 32;
   bl::k_ternarise_pack2<<<static_cast<int>(pctas), 256, 0, s>>>(W, N, K, gamma, packed);
   return launch_status();
+}
+
+int64_t bitlinear_packed3_stride(int64_t K) {
+  if (K < 1) return 0;
+  return 16 * ((((K + 4) / 5) + 15) / 16);
+}
+
+bl_status bitlinear_pack_weights3(const float* W, int64_t N, int64_t K, uint8_t* packed3,
+                                  float* gamma, void* workspace, void* stream) {
+  if (!W || !packed3 || !gamma || !workspace) return BL_ERR_INVALID_ARG;
+  if (N < 1 || K < 1) return BL_ERR_INVALID_ARG;
+  if (N > (int64_t{1} << 40) / K) return BL_ERR_UNSUPPORTED;
+  if (!aligned(W, 4) || !aligned(workspace, 8) || !aligned(gamma, 4)) return BL_ERR_ALIGNMENT;
+  int sms = 148;
+  bl_status st = device_info(&sms);
+  if (st != BL_OK) return st;
+  const cudaStream_t s = as_stream(stream);
+  auto* buckets = static_cast<unsigned long long*>(workspace);
+  bl::k_zero_u64<<<1, 256, 0, s>>>(buckets, bl::kBuckets);
+  if ((st = launch_status()) != BL_OK) return st;
+  const int64_t count = N * K;
+  int64_t ctas = (count / 4 + 255) / 256;
+  if (ctas > static_cast<int64_t>(sms) * 8) ctas = static_cast<int64_t>(sms) * 8;
+  if (ctas < 1) ctas = 1;
+  bl::k_absmean_buckets<<<static_cast<int>(ctas), 256, 0, s>>>(W, count, buckets);
+  if ((st = launch_status()) != BL_OK) return st;
+  bl::k_gamma_finalize<<<1, 32, 0, s>>>(buckets, count, gamma);
+  if ((st = launch_status()) != BL_OK) return st;
+  const int64_t S = bitlinear_packed3_stride(K);
+  int64_t pctas = (N * S + 255) / 256;
+  if (pctas > static_cast<int64_t>(sms) * 32) pctas = static_cast<int64_t>(sms) * 32;
+  bl::k_ternarise_pack3<<<static_cast<int>(pctas), 256, 0, s>>>(W, N, K, S, gamma, packed3);
+  return launch_status();
+}
+
+bl_status bitlinear_forward3(const int8_t* xq, const float* eta, const int32_t* xsum, int64_t M,
+                             int64_t K, const uint8_t* packed3, const float* gamma, int64_t N,
+                             void* y, bl_dtype ydt, int32_t* y_int, void* stream) {
+  if (M < 0 || K < 1 || N < 1) return BL_ERR_INVALID_ARG;
+  if (ydt != BL_F32 && ydt != BL_BF16) return BL_ERR_INVALID_ARG;
+  if (!packed3 || !gamma) return BL_ERR_INVALID_ARG;
+  if (M == 0) return BL_OK;
+  if (!xq || !eta || !xsum || !y) return BL_ERR_INVALID_ARG;
+  const int64_t S = bitlinear_packed3_stride(K);
+  // shared memory: the 2 KB table + 8-byte activation slots per group of five
+  // per token, kept within the 48 KB default (tokens per launch 4, 2 or 1)
+  constexpr int64_t kSmemLimit = 48 * 1024;
+  if (K > (1 << 30) || N > INT32_MAX / 2 || 2048 + S * 8 + 64 > kSmemLimit) return BL_ERR_UNSUPPORTED;
+  const int mt_max = 2048 + 4 * S * 8 + 64 <= kSmemLimit ? 4 : (2048 + 2 * S * 8 + 64 <= kSmemLimit ? 2 : 1);
+  if (!aligned(packed3, 16) || !aligned(eta, 4) || !aligned(xsum, 4) || !aligned(gamma, 4) ||
+      (y_int && !aligned(y_int, 4)) || !aligned(y, ydt == BL_F32 ? 4 : 2))
+    return BL_ERR_ALIGNMENT;
+  int sms = 148;
+  bl_status st = device_info(&sms);
+  if (st != BL_OK) return st;
+  const cudaStream_t cs = as_stream(stream);
+  const size_t esz = ydt == BL_F32 ? 4 : 2;
+  int64_t ctas = (N + bl::kG3Warps * bl::kG3Rows - 1) / (bl::kG3Warps * bl::kG3Rows);
+  if (ctas > static_cast<int64_t>(sms) * 8) ctas = static_cast<int64_t>(sms) * 8;
+  for (int64_t m0 = 0; m0 < M; m0 += mt_max) {
+    const int mc = static_cast<int>(M - m0 < mt_max ? M - m0 : mt_max);
+    const int mt = mc <= 1 ? 1 : (mc <= 2 ? 2 : 4);
+    const size_t smem = 2048 + static_cast<size_t>(mt) * S * 8 + 64;
+    const int8_t* xq_m = xq + m0 * K;
+    void* y_m = static_cast<char*>(y) + m0 * N * esz;
+    int32_t* yi_m = y_int ? y_int + m0 * N : nullptr;
+    auto go = [&](auto kern) -> bl_status {
+      static int done[kMaxDevices] = {0};
+      if (!ensure_smem(kern, 0, done)) return BL_ERR_CUDA;  // carveout only: smem <= 48 KB
+      return launch_pdl(kern, dim3(static_cast<unsigned>(ctas)), dim3(32 * bl::kG3Warps), smem, cs,
+                        xq_m, eta + m0, xsum + m0, mc, static_cast<int>(K), static_cast<int>(S),
+                        packed3, gamma, static_cast<int>(N), y_m, yi_m);
+    };
+    if (ydt == BL_F32)
+      st = mt == 1 ? go(bl::k_gemv3<1, float>) : (mt == 2 ? go(bl::k_gemv3<2, float>) : go(bl::k_gemv3<4, float>));
+    else
+      st = mt == 1 ? go(bl::k_gemv3<1, __nv_bfloat16>)
+                   : (mt == 2 ? go(bl::k_gemv3<2, __nv_bfloat16>) : go(bl::k_gemv3<4, __nv_bfloat16>));
+    if (st != BL_OK) return st;
+  }
+  return BL_OK;
 }
 
 }  // extern "C"

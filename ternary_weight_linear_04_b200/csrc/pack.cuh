@@ -172,4 +172,34 @@ __global__ void __launch_bounds__(256) k_ternarise_pack2(const float* __restrict
   }
 }
 
+// Base-3 packing of the same trits ("compact ternary packing", [Additive]
+// "Energy, Memory Bandwidth, and Serving Economics"; the layout is this
+// library's): byte g of a row = sum_j (t_{5g+j} + 1) * 3^j, j = 0..4, trits
+// past K are 0, rows of S = 16 * ceil(ceil(K/5) / 16) bytes (padding bytes
+// hold five zero trits, 121).  Same ternarisation test as k_ternarise_pack2.
+__global__ void __launch_bounds__(256) k_ternarise_pack3(const float* __restrict__ W, int64_t N,
+                                                          int64_t K, int64_t S,
+                                                          const float* __restrict__ gamma_p,
+                                                          uint8_t* __restrict__ packed3) {
+  const int64_t total = N * S;
+  const float gamma = *gamma_p;
+  for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
+       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t n = idx / S;
+    const int64_t k0 = 5 * (idx - n * S);
+    uint32_t byte = 0, pw = 1;
+#pragma unroll
+    for (int j = 0; j < 5; ++j) {
+      uint32_t digit = 1u;
+      if (k0 + j < K) {
+        const float q = __fdiv_rn(__ldg(W + n * K + k0 + j), gamma);
+        digit = (q > 0.5f) ? 2u : ((q < -0.5f) ? 0u : 1u);
+      }
+      byte += digit * pw;
+      pw *= 3u;
+    }
+    packed3[idx] = static_cast<uint8_t>(byte);
+  }
+}
+
 }  // namespace bl

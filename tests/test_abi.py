@@ -106,6 +106,18 @@ def test_bad_arguments_are_rejected_without_a_launch(L):
     assert grp(fake, 1, 1, 96, 1, arr1, arr1, n1, arr1, 1, 0, None) == _lib.BL_ERR_UNSUPPORTED  # K % 64
     assert grp(P(257), 1, 1, 64, 1, arr1, arr1, n1, arr1, 1, 0, None) == _lib.BL_ERR_ALIGNMENT
     assert grp(None, 1, 0, 64, 1, arr1, arr1, n1, arr1, 1, 0, None) == _lib.BL_OK  # M = 0
+    assert [L.bitlinear_packed3_stride(K) for K in (0, 1, 80, 81, 3200, 8192)] == [0, 16, 16, 32, 640, 1648]
+    p3 = L.bitlinear_pack_weights3
+    assert p3(None, 4, 4, fake, fake, fake, None) == _lib.BL_ERR_INVALID_ARG
+    assert p3(fake, 0, 4, fake, fake, fake, None) == _lib.BL_ERR_INVALID_ARG
+    assert p3(P(258), 4, 4, fake, fake, fake, None) == _lib.BL_ERR_ALIGNMENT
+    f3 = L.bitlinear_forward3
+    assert f3(fake, fake, fake, 1, 0, fake, fake, 8, fake, 0, None, None) == _lib.BL_ERR_INVALID_ARG
+    assert f3(fake, fake, fake, 1, 64, None, fake, 8, fake, 0, None, None) == _lib.BL_ERR_INVALID_ARG
+    assert f3(fake, fake, fake, 1, 64, fake, fake, 8, fake, 7, None, None) == _lib.BL_ERR_INVALID_ARG
+    assert f3(fake, fake, fake, 1, 1 << 20, fake, fake, 8, fake, 0, None, None) == _lib.BL_ERR_UNSUPPORTED
+    assert f3(fake, fake, fake, 1, 64, P(264), fake, 8, fake, 0, None, None) == _lib.BL_ERR_ALIGNMENT
+    assert f3(None, None, None, 0, 64, fake, fake, 8, None, 0, None, None) == _lib.BL_OK
 
 
 def test_path_selection_is_host_logic(L):

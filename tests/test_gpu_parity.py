@@ -11,6 +11,7 @@ import pytest
 import torch
 
 from oracle import native as orc
+from oracle import reference as ref
 from ternary_weight_linear_04_b200 import bitlinear as bl
 from ternary_weight_linear_04_b200 import build as libbuild
 from ternary_weight_linear_04_b200 import inputs
@@ -539,3 +540,32 @@ def test_linear_group_matches_each_matrix(M, Ns):
     ys = bl.linear_group(xd, packs, gams, out_dtype=torch.float32)
     for y, ref_y in zip(ys, refs):
         np.testing.assert_array_equal(y.cpu().numpy().view(np.uint32), ref_y.view(np.uint32))
+
+
+# ----------------------------------------------------------------- base-3 packing
+
+@pytest.mark.parametrize("N,K", [(1, 1), (7, 5), (33, 81), (130, 640), (1000, 3200), (257, 8640)])
+def test_pack3_bytes_match_the_oracle(N, K):
+    W, _ = inputs.make_case(9100 + N + K, 1, K, N)
+    t = orc.pack_weights(W, want_ternary=True)[2]
+    packed3, gamma = bl.pack_weights3(torch.from_numpy(W).cuda())
+    np.testing.assert_array_equal(packed3.cpu().numpy(), ref.pack3(t))
+    assert np.float32(gamma.cpu().numpy()[0]).view(np.uint32) == orc.pack_weights(W)[1].view(np.uint32)
+
+
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 5, 9])
+@pytest.mark.parametrize("K,N", [(64, 8), (645, 129), (3200, 1000), (8640, 333)])
+@pytest.mark.parametrize("out", ["f32", "bf16"])
+def test_forward3_matches_the_oracle(M, K, N, out):
+    """Base-3 accumulate: y_int and y bit-exact against the oracle (the same
+    values as the 2-bit path on the same trits); ragged K (a partial last
+    group and padding bytes), M above 4 (several launches)."""
+    W, x = inputs.make_case(9200 + M + K + N, M, K, N, act_dtype="bf16")
+    ref_packed, ref_gamma, t = orc.pack_weights(W, want_ternary=True)
+    ref_xq, ref_eta, ref_xsum = orc.quant_act(x)
+    ref_yint, ref_y = orc.forward(ref_xq, ref_eta, ref_packed, ref_gamma, K, N)
+    packed3, gamma = bl.pack_weights3(torch.from_numpy(W).cuda())
+    xq, eta, xsum = (torch.from_numpy(a).cuda() for a in (ref_xq, ref_eta, ref_xsum))
+    y, y_int = bl.forward3(xq, eta, xsum, packed3, gamma, N, out_dtype=DT[out], want_int=True)
+    np.testing.assert_array_equal(y_int.cpu().numpy(), ref_yint)
+    np.testing.assert_array_equal(y_bits(y.cpu()), oracle_y_bits(ref_y, out))
