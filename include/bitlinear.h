@@ -213,12 +213,15 @@ bl_status bitlinear_forward_path(const int8_t* xq, const float* eta, const int32
  *   packed, gamma, N  in   as for bitlinear_forward.
  *   y, ydt, y_int     out  as for bitlinear_forward (y_int optional).
  *   xq, eta, xsum     out  the quantised activations (M x K int8, M fp32,
- *                          M int32).  For bf16 decode batches (M <= 4,
- *                          K % 64 == 0, K * M' <= 131072 with M' = M rounded
- *                          up to 1, 2 or 4, 16-byte aligned x, packed, y) one
- *                          fused kernel runs and these are optional (NULL =
- *                          not written).  Otherwise two kernels run and they
- *                          are required scratch (BL_ERR_INVALID_ARG if NULL).
+ *                          M int32).  For bf16 decode batches of one or
+ *                          two tokens (M <= 2, K % 64 == 0, K * M' <=
+ *                          131072 with M' = M rounded up to 1 or 2, 16-byte
+ *                          aligned x, packed, y) one fused kernel runs and
+ *                          these are optional (NULL = not written).
+ *                          Otherwise two kernels run (quantiser, then the
+ *                          accumulate kernel bitlinear_forward would pick)
+ *                          and they are required scratch
+ *                          (BL_ERR_INVALID_ARG if NULL).
  *   flags             in   0 or BL_FLAG_WEIGHTS_STATIC.
  */
 bl_status bitlinear_linear(const void* x, bl_dtype xdt, int64_t M, int64_t K,

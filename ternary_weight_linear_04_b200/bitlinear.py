@@ -96,10 +96,10 @@ def forward(xq, eta, xsum, packed, gamma, N, out_dtype=torch.bfloat16, want_int=
 
 def fused_decode_ok(M, K):
     """Whether bitlinear_linear runs its single fused decode kernel for (M, K)
-    with bf16 activations (the same rule as the library; otherwise it needs
-    x~ scratch)."""
-    mt = 1 if M <= 1 else (2 if M <= 2 else 4)
-    return 1 <= M <= 4 and K >= 64 and K % 64 == 0 and K * mt <= 131072
+    with bf16 activations: one or two tokens (the same rule as the library;
+    otherwise it needs x~ scratch)."""
+    mt = 1 if M <= 1 else 2
+    return 1 <= M <= 2 and K >= 64 and K % 64 == 0 and K * mt <= 131072
 
 
 DECODE_SHAPE_FIELDS = ("team_warps", "rows_per_block", "teams", "words_per_lane", "rows_per_cta",

@@ -28,6 +28,7 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 constexpr int kGemvMaxM = 4;  // largest token count the CUDA-core decode kernel takes
+constexpr int kFusedMaxM = 2;  // largest token count bitlinear_linear fuses into one kernel
 
 // Tokens rounded up to the decode kernel's widths (1, 2, 4).
 inline int decode_mt(int64_t M) { return M <= 1 ? 1 : (M <= 2 ? 2 : 4); }
@@ -854,7 +855,11 @@ bl_status bitlinear_linear(const void* x, bl_dtype xdt, int64_t M, int64_t K, co
   if (M == 0) return BL_OK;
   if (!x || !y) return BL_ERR_INVALID_ARG;
   if (127 * K >= (int64_t{1} << 31)) return BL_ERR_UNSUPPORTED;
-  const bool fused = decode_ok(M, K) && xdt == BL_BF16 &&
+  // One fused kernel for one or two tokens; from three tokens on, the fused
+  // kernel's per-CTA quantiser (every CTA quantises all M rows) costs more
+  // than the separate quantiser kernel (measured: M = 4, K = 8640 fused
+  // 17.6 us against 4.5 + 8.3 us), so two kernels run.
+  const bool fused = M <= kFusedMaxM && decode_ok(M, K) && xdt == BL_BF16 &&
                      aligned(x, 16) && aligned(packed, 16) && aligned(y, 16) &&
                      (!y_int || aligned(y_int, 16)) && (!xq || aligned(xq, 16)) &&
                      (!eta || aligned(eta, 4)) && (!xsum || aligned(xsum, 4)) && N <= INT32_MAX / 2;

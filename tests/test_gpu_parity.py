@@ -406,6 +406,10 @@ def test_decode_forced_shapes(forced_shape, M, RB, G, K, N):
     ref_xq, ref_eta, ref_xsum = orc.quant_act(x)
     ref_yint, ref_y = orc.forward(ref_xq, ref_eta, ref_packed, ref_gamma, K, N)
     xd = torch.from_numpy(x).cuda().to(torch.bfloat16)
+    # the fused kernel at every M (a one-matrix group always fuses)
+    (yg,) = bl.linear_group(xd, [packed], [gamma], out_dtype=torch.bfloat16, weights_static=True)
+    np.testing.assert_array_equal(y_bits(yg.cpu()), orc.f32_to_bf16_bits(ref_y))
+    # bitlinear_linear (fused for M <= 2) with its optional outputs
     y, (xq, eta, xsum), y_int = bl.linear(xd, packed, gamma, N, out_dtype=torch.bfloat16,
                                           want_quant=True, want_int=True, weights_static=True)
     np.testing.assert_array_equal(xq.cpu().numpy(), ref_xq)
