@@ -247,6 +247,14 @@ bl_status bitlinear_linear(const void* x, bl_dtype xdt, int64_t M, int64_t K,
 bl_status bitlinear_decode_shape(int64_t M, int64_t K, int64_t N, int fused, int32_t* shape);
 
 /*
+ * The same for a GPU with `sms` SMs, without querying a device (host logic
+ * only; usable without a GPU).  Errors as above, plus BL_ERR_INVALID_ARG for
+ * sms < 1.
+ */
+bl_status bitlinear_decode_shape_for(int64_t M, int64_t K, int64_t N, int fused, int sms,
+                                     int32_t* shape);
+
+/*
  * Force the decode kernel's shape for every later launch in this process:
  * team_warps G in 1..16 and rows_per_block RB in {1, 2, 4, 8, 16} (RB * M'
  * <= 16 with M' = M rounded up to 1, 2 or 4); 0 for either leaves that

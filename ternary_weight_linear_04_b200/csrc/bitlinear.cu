@@ -580,6 +580,25 @@ bl_status bitlinear_linear_group(const void* x, bl_dtype xdt, int64_t M, int64_t
                        : launch_decode<__nv_bfloat16, __nv_bfloat16>(a, sms, cs);
 }
 
+bl_status bitlinear_decode_shape_for(int64_t M, int64_t K, int64_t N, int fused, int sms,
+                                     int32_t* shape) {
+  if (!shape || N < 1 || sms < 1) return BL_ERR_INVALID_ARG;
+  if (!decode_ok(M, K) || N > INT32_MAX / 2) return BL_ERR_UNSUPPORTED;
+  DecGeom g;
+  if (!decode_geometry(decode_mt(M), M, K, N, sms, fused ? 2 : 1, &g)) return BL_ERR_UNSUPPORTED;
+  shape[0] = g.G;
+  shape[1] = g.RB;
+  shape[2] = g.teams;
+  shape[3] = g.nwj;
+  shape[4] = g.rows_per_cta;
+  shape[5] = g.grid;
+  shape[6] = g.bpc;
+  shape[7] = g.stages;
+  shape[8] = g.x_staged;
+  shape[9] = static_cast<int32_t>(g.smem);
+  return BL_OK;
+}
+
 bl_status bitlinear_decode_shape(int64_t M, int64_t K, int64_t N, int fused, int32_t* shape) {
   if (!shape || N < 1) return BL_ERR_INVALID_ARG;
   if (!decode_ok(M, K) || N > INT32_MAX / 2) return BL_ERR_UNSUPPORTED;

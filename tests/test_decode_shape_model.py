@@ -1,0 +1,83 @@
+"""The decode kernel's launch-shape model is host logic: checked here on the
+CPU (no GPU) through bitlinear_decode_shape_for with B200's 148 SMs.
+
+Invariants every shape must keep (the kernel relies on them), and the
+shapes the model picks for the decode_3b matrices, which a forced-shape
+sweep on the GPU measured as the fastest.
+"""
+import ctypes
+
+import pytest
+
+from ternary_weight_linear_04_b200 import _lib
+from ternary_weight_linear_04_b200 import build as libbuild
+
+FIELDS = ("G", "RB", "teams", "nwj", "rpc", "grid", "bpc", "stages", "x_staged", "smem")
+
+
+@pytest.fixture(scope="module")
+def L():
+    libbuild.build()
+    return _lib.lib()
+
+
+def shape(L, M, K, N, fused=1, sms=148):
+    buf = (ctypes.c_int32 * 10)()
+    st = L.bitlinear_decode_shape_for(M, K, N, fused, sms, buf)
+    return st, dict(zip(FIELDS, list(buf)))
+
+
+SHAPES = [(M, K, N) for M in (1, 2, 3, 4)
+          for K, N in ((64, 5), (256, 256), (3200, 8640), (8640, 3200), (8192, 8192), (8192, 1024),
+                       (8192, 28672), (28672, 8192), (4096, 11008), (16384, 77))]
+
+
+@pytest.mark.parametrize("M,K,N", SHAPES)
+def test_shape_invariants(L, M, K, N):
+    mt = 1 if M == 1 else (2 if M == 2 else 4)
+    st, g = shape(L, M, K, N)
+    if K * mt > 131072:
+        assert st == _lib.BL_ERR_UNSUPPORTED
+        return
+    assert st == _lib.BL_OK, st
+    assert 1 <= g["G"] <= 16 and g["teams"] == 16 // g["G"]
+    assert g["RB"] in (1, 2, 4, 8, 16) and g["RB"] * mt <= 16
+    assert 32 * g["G"] * g["nwj"] >= K // 16                  # every packed word has a lane
+    assert g["rpc"] * g["grid"] >= N and (g["grid"] - 1) * g["rpc"] < N
+    assert g["grid"] <= max(148, N)
+    blocks = -(-g["rpc"] // g["RB"])
+    if g["G"] > 1:
+        assert blocks <= 64                                   # reduction slots per CTA
+    assert 1 <= g["bpc"] <= blocks and 1 <= g["stages"] <= 8
+    assert g["smem"] <= 227 * 1024
+    # shared memory = x~ slots + staged activations + ring + tail, all accounted for
+    slots = mt * 32 * g["G"] * g["nwj"] * 16
+    ring = g["stages"] * g["bpc"] * g["RB"] * (K // 4)
+    assert g["smem"] >= slots + ring
+    if g["x_staged"]:
+        assert g["smem"] >= slots + ring + M * K * 2
+
+
+def test_decode_3b_shapes_are_the_measured_best(L):
+    """A forced-shape sweep on B200 measured G=1, RB=4 (K=3200) and G=1,
+    RB=2 (K=8640) as the fastest for one token; the model picks them."""
+    _, a = shape(L, 1, 3200, 8640)
+    _, b = shape(L, 1, 8640, 3200)
+    assert (a["G"], a["RB"]) == (1, 4) and (b["G"], b["RB"]) == (1, 2)
+    # and the whole share of a CTA fits the ring: the weights are prefetched
+    assert a["bpc"] * a["stages"] * a["RB"] >= a["rpc"]
+    assert b["bpc"] * b["stages"] * b["RB"] >= b["rpc"]
+
+
+def test_fewer_sms_more_rows_per_cta(L):
+    _, a = shape(L, 1, 3200, 8640, sms=148)
+    _, b = shape(L, 1, 3200, 8640, sms=74)
+    assert b["rpc"] > a["rpc"] and b["grid"] <= 74
+
+
+def test_bad_arguments(L):
+    assert shape(L, 1, 3200, 8640, sms=0)[0] == _lib.BL_ERR_INVALID_ARG
+    assert shape(L, 1, 3200, 0)[0] == _lib.BL_ERR_INVALID_ARG
+    assert shape(L, 5, 3200, 8640)[0] == _lib.BL_ERR_UNSUPPORTED
+    buf = (ctypes.c_int32 * 10)()
+    assert L.bitlinear_decode_shape_for(1, 3200, 8640, 1, 148, None) == _lib.BL_ERR_INVALID_ARG
