@@ -17,6 +17,9 @@ Citations (page title tags as in ``bitlinear_oracle.c``):
   2-bit codes and bit order -- [Production] "Production Deployment Standards"
                                guideline 1; [No-Multiply] "Kernel
                                Implementation: The Lookup Table Approach"
+  RMSNorm before the quant  -- [Production] "2. Absmax Dynamic Activation
+                               Quantization" (normalised first, no affine),
+                               BitLinear158.forward (rsqrt(mean(x^2) + 1e-6))
   base-3 packing            -- [Additive] "Energy, Memory Bandwidth, and
                                Serving Economics" (compact ternary packing,
                                named only: the layout is this build's
@@ -128,6 +131,36 @@ def forward3(xq, eta, packed3, gamma, K):
     t = unpack3(packed3, K)
     y_int = accumulate(xq, t)
     return y_int, rescale(y_int, eta, gamma)
+
+
+RMS_EPS = np.float32(1e-6)
+
+
+def rmsnorm(x):
+    """RMSNorm without affine parameters, before the quantiser ([Production]
+    "2. Absmax Dynamic Activation Quantization" and BitLinear158.forward:
+    norm = rsqrt(mean(x^2) + 1e-6), x_norm = x * norm), per token.
+    Readings: mean(x^2) = RN32(RN64(exact sum of x^2) / K) with the
+    division in fp64 (the sum order is unspecified on the pages; the exact
+    sum makes it order-free, as for gamma); rsqrt(v) = RN32(1 / RN32(sqrt(v)))
+    (an IEEE fp32 square root, then an IEEE fp32 division); every other step
+    one fp32 rounding."""
+    x = np.asarray(x, dtype=np.float32)
+    M, K = x.shape
+    out = np.empty_like(x)
+    for m in range(M):
+        S = math.fsum(float(v) * float(v) for v in x[m])   # squares exact in fp64; fsum = RN64 of the exact sum
+        ms = np.float32(S / K)                               # fp64 division, then RN32
+        v = np.float32(ms + RMS_EPS)
+        s = np.sqrt(v, dtype=np.float32)                     # IEEE fp32 square root
+        r = np.float32(1.0) / s                              # IEEE fp32 division
+        out[m] = x[m] * r
+    return out
+
+
+def rmsnorm_quant_act(x):
+    """RMSNorm then the per-token absmax int8 quantiser: (x~, eta, xsum)."""
+    return quant_act(rmsnorm(x))
 
 
 def pack_weights(W):
