@@ -153,6 +153,31 @@ bl_status bitlinear_quant_act(const void* x, bl_dtype xdt, int64_t M, int64_t K,
                               int8_t* xq, float* eta, int32_t* xsum, void* stream);
 
 /*
+ * RMSNorm without affine parameters, fused with the per-token quantiser.
+ * [Production] "2. Absmax Dynamic Activation Quantization" (the activations
+ * are RMS-normalised before absmax quantisation) and BitLinear158.forward
+ * (norm = rsqrt(mean(x^2) + 1e-6), x_norm = x * norm), per token:
+ *   mean  = RN32(RN64(exact sum_k x^2) / K)   (the division in fp64)
+ *   r     = RN32(1 / RN32(sqrt(RN32(mean + 1e-6))))
+ *   x_norm = RN32(x * r), then bitlinear_quant_act's rule on x_norm.
+ * The sum of squares is formed exactly, so the result does not depend on
+ * the summation order and is identical on every device.
+ *
+ *   x     in   M x K row-major, bf16 (xdt = BL_BF16).
+ *   M     in   tokens >= 0 (M = 0 is a no-op returning BL_OK; the M-sized
+ *              buffers may then be NULL).
+ *   K     in   in_features, 1 <= K <= 2^24.
+ *   xq    out  int8, M x K row-major: the codes of x_norm.
+ *   eta   out  fp32, M: max(max_k |x_norm[m,k]|, 1e-5).
+ *   xsum  out  int32, M: sum_k xq[m,k].
+ * Errors: BL_ERR_INVALID_ARG for null pointers, M < 0, K < 1 or an unknown
+ * dtype; BL_ERR_UNSUPPORTED for fp32 x or K > 2^24; BL_ERR_ALIGNMENT if x is
+ * not 2-byte aligned or eta/xsum not 4-byte aligned.
+ */
+bl_status bitlinear_rmsnorm_quant_act(const void* x, bl_dtype xdt, int64_t M, int64_t K,
+                                      int8_t* xq, float* eta, int32_t* xsum, void* stream);
+
+/*
  * Per-token half of the layer: integer accumulation and rescale.
  * [Production] "The MatMul-Free Breakthrough" (add where W~ = +1, subtract
  * where W~ = -1, skip zeros), [Additive] "3. Additive Integer Accumulation",

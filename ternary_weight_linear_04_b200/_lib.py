@@ -27,6 +27,7 @@ SIGNATURES = {
     "bitlinear_pack_weights": (_I, [_P, _I64, _I64, _P, _P, _P, _P]),
     "bitlinear_pack_weights_noalloc": (_I, [_P, _I64, _I64, _P, _P, _P]),
     "bitlinear_quant_act": (_I, [_P, _I, _I64, _I64, _P, _P, _P, _P]),
+    "bitlinear_rmsnorm_quant_act": (_I, [_P, _I, _I64, _I64, _P, _P, _P, _P]),
     "bitlinear_forward": (_I, [_P, _P, _P, _I64, _I64, _P, _P, _I64, _P, _I, _P, _P]),
     "bitlinear_forward_path": (_I, [_P, _P, _P, _I64, _I64, _P, _P, _I64, _P, _I, _P, _I,
                                     ctypes.c_uint, _P]),

@@ -73,6 +73,26 @@ def quant_act(x, stream=None, out=None):
     return xq, eta, xsum
 
 
+def rmsnorm_quant_act(x, stream=None, out=None):
+    """RMSNorm (no affine, eps 1e-6) fused with the per-token quantiser.
+    Activations (M x K, bf16, CUDA) -> (xq int8 M x K, eta fp32 M, xsum int32 M)
+    of the normalised rows."""
+    _require_cuda(x)
+    if x.dim() != 2 or x.dtype != torch.bfloat16:
+        raise ValueError("x must be a 2-D bfloat16 tensor")
+    M, K = x.shape
+    dev = x.device
+    if out is None:
+        out = (torch.empty((M, K), dtype=torch.int8, device=dev),
+               torch.empty(M, dtype=torch.float32, device=dev),
+               torch.empty(M, dtype=torch.int32, device=dev))
+    xq, eta, xsum = out
+    check(_lib.lib().bitlinear_rmsnorm_quant_act(_ptr(x), _DTYPES[x.dtype], M, K, _ptr(xq),
+                                                 _ptr(eta), _ptr(xsum), _stream(stream)),
+          "bitlinear_rmsnorm_quant_act")
+    return xq, eta, xsum
+
+
 def forward(xq, eta, xsum, packed, gamma, N, out_dtype=torch.bfloat16, want_int=False,
             path="auto", stream=None, out=None, out_int=None, weights_static=False):
     """Integer accumulation + rescale.  Returns y (M x N), or (y, y_int) if want_int.

@@ -23,6 +23,7 @@
 #include "gemv.cuh"
 #include "pack.cuh"
 #include "quant.cuh"
+#include "rmsnorm.cuh"
 
 namespace {
 
@@ -670,6 +671,26 @@ bl_status bitlinear_pack_weights(const float* W, int64_t N, int64_t K, uint8_t* 
   if (pctas > static_cast<int64_t>(sms) * 32) pctas = static_cast<int64_t>(sms) * 32;
   bl::k_ternarise_pack2<<<static_cast<int>(pctas), 256, 0, s>>>(W, N, K, gamma, packed);
   return launch_status();
+}
+
+bl_status bitlinear_rmsnorm_quant_act(const void* x, bl_dtype xdt, int64_t M, int64_t K,
+                                      int8_t* xq, float* eta, int32_t* xsum, void* stream) {
+  if (M < 0 || K < 1 || (xdt != BL_F32 && xdt != BL_BF16)) return BL_ERR_INVALID_ARG;
+  if (M == 0) return BL_OK;
+  if (!x || !xq || !eta || !xsum) return BL_ERR_INVALID_ARG;
+  if (xdt != BL_BF16) return BL_ERR_UNSUPPORTED;  // the exact sum of squares needs bf16 inputs
+  if (K > (int64_t{1} << 24)) return BL_ERR_UNSUPPORTED;  // keeps xsum within int32
+  if (!aligned(x, 2) || !aligned(eta, 4) || !aligned(xsum, 4)) return BL_ERR_ALIGNMENT;
+  int sms = 148;
+  bl_status st = device_info(&sms);
+  if (st != BL_OK) return st;
+  static int carve_done[kMaxDevices] = {0};
+  if (!ensure_smem(bl::k_rmsnorm_quant, 0, carve_done)) return BL_ERR_CUDA;
+  const int64_t ctas = M < static_cast<int64_t>(sms) * 8 ? M : static_cast<int64_t>(sms) * 8;
+  const int vec = (K % 8 == 0 && aligned(x, 16) && aligned(xq, 8)) ? 1 : 0;
+  return launch_pdl(bl::k_rmsnorm_quant, dim3(static_cast<unsigned>(ctas)), dim3(256), 0,
+                    as_stream(stream), static_cast<const __nv_bfloat16*>(x), M, K, vec, xq, eta,
+                    xsum);
 }
 
 int64_t bitlinear_packed3_stride(int64_t K) {

@@ -27,15 +27,11 @@ __global__ void k_zero_u64(unsigned long long* p, int n) {
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) p[i] = 0;
 }
 
-// Adds one fp32 bit pattern per lane into the CTA's shared buckets.  All 32
-// lanes must call it together (lanes with nothing to add pass u = 0).  Lanes
-// that share a bucket are summed with one warp reduction and a single shared
+// sb[b] += m for one (bucket b, integer m < 2^24) per lane.  All 32 lanes
+// must call it together (lanes with nothing to add pass m = 0).  Lanes that
+// share a bucket are summed with one warp reduction and a single shared
 // atomic, one distinct bucket per loop trip.
-__device__ __forceinline__ void bucket_add_warp(unsigned long long* sb, uint32_t u) {
-  const uint32_t e = (u >> 23) & 0xFFu;
-  const uint32_t frac = u & 0x7FFFFFu;
-  const uint32_t b = e ? e : 1u;                  // subnormals share bucket 1
-  const uint32_t m = e ? (frac | 0x800000u) : frac;
+__device__ __forceinline__ void bucket_add_warp_bm(unsigned long long* sb, uint32_t b, uint32_t m) {
   const int lane = threadIdx.x & 31;
   unsigned todo = 0xFFFFFFFFu;
   while (todo) {
@@ -47,6 +43,16 @@ __device__ __forceinline__ void bucket_add_warp(unsigned long long* sb, uint32_t
     if (lane == leader && s) atomicAdd(&sb[lb], static_cast<unsigned long long>(s));
     todo &= ~grp;
   }
+}
+
+// Adds one fp32 bit pattern per lane: bucket = biased exponent, m = integer
+// mantissa (|W| = m * 2^(b-150)).
+__device__ __forceinline__ void bucket_add_warp(unsigned long long* sb, uint32_t u) {
+  const uint32_t e = (u >> 23) & 0xFFu;
+  const uint32_t frac = u & 0x7FFFFFu;
+  const uint32_t b = e ? e : 1u;                  // subnormals share bucket 1
+  const uint32_t m = e ? (frac | 0x800000u) : frac;
+  bucket_add_warp_bm(sb, b, m);
 }
 
 // buckets[b] += sum of the integer mantissas m of all |W| with bucket b.

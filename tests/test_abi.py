@@ -61,6 +61,16 @@ def test_bad_arguments_are_rejected_without_a_launch(L):
     assert L.bitlinear_quant_act(fake, 0, 1, 0, fake, fake, fake, None) == _lib.BL_ERR_INVALID_ARG
     assert L.bitlinear_quant_act(P(257), 1, 1, 4, fake, fake, fake, None) == _lib.BL_ERR_ALIGNMENT
     assert L.bitlinear_quant_act(fake, 0, 0, 4, fake, fake, fake, None) == _lib.BL_OK  # M = 0: no-op
+    rq = L.bitlinear_rmsnorm_quant_act
+    assert rq(None, 1, 1, 4, fake, fake, fake, None) == _lib.BL_ERR_INVALID_ARG
+    assert rq(None, 1, 0, 4, None, None, None, None) == _lib.BL_OK
+    assert rq(fake, 7, 1, 4, fake, fake, fake, None) == _lib.BL_ERR_INVALID_ARG
+    assert rq(fake, 1, -1, 4, fake, fake, fake, None) == _lib.BL_ERR_INVALID_ARG
+    assert rq(fake, 1, 1, 0, fake, fake, fake, None) == _lib.BL_ERR_INVALID_ARG
+    assert rq(fake, 0, 1, 4, fake, fake, fake, None) == _lib.BL_ERR_UNSUPPORTED  # fp32 input
+    assert rq(fake, 1, 1, (1 << 24) + 1, fake, fake, fake, None) == _lib.BL_ERR_UNSUPPORTED
+    assert rq(P(257), 1, 1, 4, fake, fake, fake, None) == _lib.BL_ERR_ALIGNMENT
+    assert rq(fake, 1, 1, 4, fake, P(258), fake, None) == _lib.BL_ERR_ALIGNMENT
     fwd = L.bitlinear_forward
     assert fwd(None, fake, fake, 1, 64, fake, fake, 8, fake, 0, None, None) == _lib.BL_ERR_INVALID_ARG
     assert fwd(fake, fake, fake, 1, 0, fake, fake, 8, fake, 0, None, None) == _lib.BL_ERR_INVALID_ARG

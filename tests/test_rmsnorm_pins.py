@@ -73,3 +73,9 @@ def test_planted_mistakes_fail():
     # sum instead of mean
     bad2 = x[0] / np.sqrt(np.float32(np.sum(x[0].astype(np.float64) ** 2)) + np.float32(1e-6))
     assert ulps(bad2, exact).max() > 4
+    # eps 1e-5 (the quantisers' floor) in place of 1e-6
+    bad3 = x[0] / np.sqrt(np.float32(np.mean(x[0].astype(np.float64) ** 2)) + np.float32(1e-5))
+    assert ulps(bad3, exact).max() > 4
+    # mean over K - 1 values
+    bad4 = x[0] / np.sqrt(np.float32(np.sum(x[0].astype(np.float64) ** 2) / 256) + np.float32(1e-6))
+    assert ulps(bad4, exact).max() > 4
