@@ -164,12 +164,16 @@ class Capture:
 
 def timed(fn_replays, stream, world):
     """Device time of fn_replays(): events recorded on `stream`, and the work
-    (graph replays, library calls) issued on that same stream."""
+    (graph replays, library calls) issued on that same stream.  A short sleep
+    kernel ahead of the start event keeps the stream busy while the host
+    enqueues the work, so no host-submission gap falls inside a short timed
+    region."""
     barrier(world)
     torch.cuda.synchronize()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
+        torch.cuda._sleep(200000)  # about 0.1 ms, before the start event
         t0.record(stream)
         fn_replays()
         t1.record(stream)
@@ -243,10 +247,12 @@ def run_ours(args, world, rank, local):
     full, rem = divmod(args.steps, G)
     g_full = Capture([fn for c in range(G) for fn in step_calls(c)], stream)
     g_rem = Capture([fn for c in range(rem) for fn in step_calls(c)], stream) if rem else None
-    # graph warm-up
+    # graph warm-up (both graphs: a graph's first replay uploads it)
     with torch.cuda.stream(stream):
         for _ in range(2):
             g_full.replay()
+            if g_rem:
+                g_rem.replay()
     torch.cuda.synchronize()
 
     def replays():
@@ -293,7 +299,7 @@ def run_ours(args, world, rank, local):
            "clocks": clk.summary()}
 
     sections = (set(args.sections.split(",")) if args.sections else
-                {"e2e", "prefill", "pack", "sweep", "layer70b", "crossover", "base3"})
+                {"e2e", "prefill", "pack", "sweep", "layer70b", "crossover", "base3", "rmsnorm"})
     if args.quick:
         sections = set()
     if "e2e" in sections:
@@ -314,6 +320,8 @@ def run_ours(args, world, rank, local):
         out["crossover"] = run_crossover(dev, stream, world, peaks, l2)
     if "base3" in sections:
         out["base3"] = run_base3(dev, stream, world, peaks, l2)
+    if "rmsnorm" in sections:
+        out["rmsnorm"] = run_rmsnorm(dev, stream, world, peaks, l2)
     if (rank == 0) and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = run_cpu_baseline(args.cpu_seconds)
     return out
@@ -680,6 +688,56 @@ def run_base3(dev, stream, world, peaks, l2):
             "rows": rows}
 
 
+def run_rmsnorm(dev, stream, world, peaks, l2):
+    """Fused RMSNorm + quantiser (bitlinear_rmsnorm_quant_act) against the
+    plain quantiser (bitlinear_quant_act), bf16 rows; algorithmic bytes =
+    2MK read + MK codes + 8M (eta, xsum) written."""
+    from ternary_weight_linear_04_b200 import _lib, inputs
+    L = _lib.lib()
+    P = ctypes.c_void_p
+    sptr = ctypes.c_void_p(stream.cuda_stream)
+    hbm = float(peaks["hbm_gbs"])
+    rng = np.random.default_rng(9)
+    rows = []
+    for M, K in ((1, 3200), (1, 8640), (64, 3200), (2048, 3200), (2048, 8640)):
+        copies = max(1, min(64, int(np.ceil(3 * l2 / (2 * M * K)))))
+        x0 = torch.from_numpy(inputs.draw_activations(rng, M, K, "normal", "bf16"))
+        bufs = []
+        for _ in range(copies):
+            bufs.append(dict(x=x0.to(dev).to(torch.bfloat16),
+                             xq=torch.empty((M, K), dtype=torch.int8, device=dev),
+                             eta=torch.empty(M, dtype=torch.float32, device=dev),
+                             xsum=torch.empty(M, dtype=torch.int32, device=dev)))
+        torch.cuda.synchronize()
+        res = {"M": M, "K": K, "copies": copies}
+        nbytes = 3 * M * K + 8 * M
+        for name, fn in (("rmsnorm_quant", L.bitlinear_rmsnorm_quant_act),
+                         ("quant_only", L.bitlinear_quant_act)):
+            calls = [lambda b=b, fn=fn: _chk(fn(P(b["x"].data_ptr()), _lib.BL_BF16, M, K,
+                                               P(b["xq"].data_ptr()), P(b["eta"].data_ptr()),
+                                               P(b["xsum"].data_ptr()), sptr), name)
+                     for b in bufs]
+            with torch.cuda.stream(stream):
+                for c in calls:
+                    c()
+            torch.cuda.synchronize()
+            gr = Capture(calls, stream)
+            with torch.cuda.stream(stream):
+                gr.replay()
+            torch.cuda.synchronize()
+            reps = max(3, 200 // copies)
+            t = max_over_ranks(timed(lambda: [gr.replay() for _ in range(reps)], stream, world),
+                               world) / (reps * copies)
+            res[name] = {"us": round(t * 1e6, 2), "gbs": round(nbytes / t / 1e9, 1),
+                         "hbm_frac": round(nbytes / t / 1e9 / hbm, 4)}
+        rows.append(res)
+        del bufs
+        torch.cuda.empty_cache()
+    return {"what": "RMSNorm (exact sum of squares) fused with the quantiser vs. the quantiser "
+                    "alone; inputs rotate over copies (> 3x L2 where the rows allow, else "
+                    "L2-resident, as in decode)", "rows": rows}
+
+
 def run_pack(mats, stream, world):
     from ternary_weight_linear_04_b200 import bitlinear as bl
     m = mats[0]
@@ -795,7 +853,8 @@ def main():
     ap.add_argument("--m", type=int, default=1, help="tokens per step (decode batch)")
     ap.add_argument("--quick", action="store_true", help="headline only (no e2e/prefill/pack)")
     ap.add_argument("--sections", default="",
-                    help="comma list of extra sections: e2e,prefill,pack,sweep,layer70b,crossover,base3")
+                    help="comma list of extra sections: e2e,prefill,pack,sweep,layer70b,crossover,base3,"
+                         "rmsnorm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-seconds", type=float, default=120.0,
