@@ -107,6 +107,49 @@ bl_status bitlinear_pack_weights(const float* W, int64_t N, int64_t K,
                                  void* workspace, void* stream);
 
 /*
+ * The three steps of bitlinear_pack_weights as separate calls, for a weight
+ * matrix split by rows over several GPUs (each holding rows [n0, n1)).
+ * gamma is a mean over the WHOLE matrix ([Production] "1. Absmean Weight
+ * Quantization"), so every shard must ternarise with the same gamma: each
+ * GPU forms the exact bucket sums of its own rows, the buckets are summed
+ * over the GPUs as 64-bit integers (an all-reduce; integer addition makes the
+ * result independent of the order and the number of shards), and every GPU
+ * derives the identical gamma from the totals.  pack_weights(W) equals
+ * absmean_buckets(W) -> gamma_from_buckets(count = N*K) -> ternarise_pack,
+ * and on any row split the shards' packed bytes and gamma are bit-identical
+ * to those of the whole matrix.
+ *
+ * Bucket layout: 256 uint64 (bitlinear_pack_workspace_bytes(), 8-byte
+ * aligned).  Bucket b (1..254) holds the sum of the integer significands m
+ * (< 2^24) of every |W| = m * 2^(b-150), b the biased fp32 exponent
+ * (subnormals in bucket 1).  Buckets 0 and 255 hold no finite values
+ * (NaN/Inf weights are outside the contract).  Two's-complement int64
+ * addition of the buckets (what an int64 sum all-reduce does) gives the
+ * same totals as unsigned addition.
+ */
+
+/* Step 1: zero `buckets`, then add the shard's |W| (fp32, N x K row-major,
+ * N*K < 2^40).  Errors as bitlinear_pack_weights (buckets in place of
+ * workspace). */
+bl_status bitlinear_absmean_buckets(const float* W, int64_t N, int64_t K, void* buckets,
+                                    void* stream);
+
+/* Step 2: gamma = max(RN32(RN64(S) / count), 1e-5), S the exact total the
+ * buckets hold and count >= 1 the number of elements of the whole matrix
+ * (<= 2^40).  One fp32 written on the device.  Errors: BL_ERR_INVALID_ARG for
+ * null pointers or count < 1; BL_ERR_UNSUPPORTED for count > 2^40;
+ * BL_ERR_ALIGNMENT if buckets is not 8-byte or gamma not 4-byte aligned. */
+bl_status bitlinear_gamma_from_buckets(const void* buckets, int64_t count, float* gamma,
+                                       void* stream);
+
+/* Step 3: ternarise rows of W (N x K) with the given device gamma and pack
+ * them as bitlinear_pack_weights does (N x ceil(K/4) bytes).  Errors:
+ * BL_ERR_INVALID_ARG for null pointers or N, K < 1; BL_ERR_UNSUPPORTED for
+ * N*K >= 2^40; BL_ERR_ALIGNMENT if W or gamma is not 4-byte aligned. */
+bl_status bitlinear_ternarise_pack(const float* W, int64_t N, int64_t K, const float* gamma,
+                                   uint8_t* packed, void* stream);
+
+/*
  * bitlinear_pack_weights for callers that cannot allocate device memory:
  * for example a library running inside a host framework that owns every
  * byte of device memory through its own pool, or a latency-critical path

@@ -25,6 +25,9 @@ SIGNATURES = {
     "bitlinear_packed_bytes": (ctypes.c_size_t, [_I64, _I64]),
     "bitlinear_pack_workspace_bytes": (ctypes.c_size_t, []),
     "bitlinear_pack_weights": (_I, [_P, _I64, _I64, _P, _P, _P, _P]),
+    "bitlinear_absmean_buckets": (_I, [_P, _I64, _I64, _P, _P]),
+    "bitlinear_gamma_from_buckets": (_I, [_P, _I64, _P, _P]),
+    "bitlinear_ternarise_pack": (_I, [_P, _I64, _I64, _P, _P, _P]),
     "bitlinear_pack_weights_noalloc": (_I, [_P, _I64, _I64, _P, _P, _P]),
     "bitlinear_quant_act": (_I, [_P, _I, _I64, _I64, _P, _P, _P, _P]),
     "bitlinear_rmsnorm_quant_act": (_I, [_P, _I, _I64, _I64, _P, _P, _P, _P]),

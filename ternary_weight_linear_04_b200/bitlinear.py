@@ -56,6 +56,45 @@ def pack_weights(W, stream=None, workspace=None, packed=None, gamma=None):
     return packed, gamma
 
 
+def absmean_buckets(W, stream=None, out=None):
+    """Exact |W| exponent buckets of a row shard (fp32 N x K, CUDA) -> int64[256]
+    (uint64 totals in two's complement; sum them over shards with an int64
+    all-reduce)."""
+    _require_cuda(W)
+    if W.dtype != torch.float32 or W.dim() != 2:
+        raise ValueError("W must be a 2-D float32 tensor")
+    N, K = W.shape
+    b = out if out is not None else torch.empty(256, dtype=torch.int64, device=W.device)
+    check(_lib.lib().bitlinear_absmean_buckets(_ptr(W), N, K, _ptr(b), _stream(stream)),
+          "bitlinear_absmean_buckets")
+    return b
+
+
+def gamma_from_buckets(buckets, count, stream=None, out=None):
+    """gamma (fp32[1]) from bucket totals of a whole matrix of `count` elements."""
+    _require_cuda(buckets)
+    if buckets.dtype != torch.int64 or buckets.numel() != 256:
+        raise ValueError("buckets must be 256 int64 values")
+    g = out if out is not None else torch.empty(1, dtype=torch.float32, device=buckets.device)
+    check(_lib.lib().bitlinear_gamma_from_buckets(_ptr(buckets), int(count), _ptr(g),
+                                                  _stream(stream)), "bitlinear_gamma_from_buckets")
+    return g
+
+
+def ternarise_pack(W, gamma, stream=None, out=None):
+    """Rows of W (fp32 N x K, CUDA) ternarised with a given gamma and packed
+    (uint8 N x ceil(K/4))."""
+    _require_cuda(W, gamma)
+    if W.dtype != torch.float32 or W.dim() != 2:
+        raise ValueError("W must be a 2-D float32 tensor")
+    N, K = W.shape
+    p = out if out is not None else torch.empty((N, (K + 3) // 4), dtype=torch.uint8,
+                                                 device=W.device)
+    check(_lib.lib().bitlinear_ternarise_pack(_ptr(W), N, K, _ptr(gamma), _ptr(p), _stream(stream)),
+          "bitlinear_ternarise_pack")
+    return p
+
+
 def quant_act(x, stream=None, out=None):
     """Activations (M x K, fp32 or bf16, CUDA) -> (xq int8 M x K, eta fp32 M, xsum int32 M)."""
     _require_cuda(x)

@@ -41,7 +41,7 @@ __global__ void __launch_bounds__(32 * kG3Warps) k_gemv3(
     int M, int K, int S, const uint8_t* __restrict__ packed3, const float* __restrict__ gamma_p,
     int N, void* __restrict__ y, int32_t* __restrict__ y_int) {
   constexpr int V = kG3Rows * MT;
-  extern __shared__ __align__(16) uint8_t smem[];
+  extern __shared__ __align__(128) uint8_t smem[];
   uint2* lut = reinterpret_cast<uint2*>(smem);             // 256 entries
   uint2* xs = reinterpret_cast<uint2*>(smem + 256 * 8);    // [MT][S] activation slots
   float* s_scale = reinterpret_cast<float*>(xs + MT * S);

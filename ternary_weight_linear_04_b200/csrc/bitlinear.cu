@@ -645,32 +645,67 @@ size_t bitlinear_packed_bytes(int64_t N, int64_t K) {
 
 size_t bitlinear_pack_workspace_bytes(void) { return bl::kBuckets * sizeof(unsigned long long); }
 
+bl_status bitlinear_absmean_buckets(const float* W, int64_t N, int64_t K, void* buckets,
+                                   void* stream) {
+  if (!W || !buckets) return BL_ERR_INVALID_ARG;
+  if (N < 1 || K < 1) return BL_ERR_INVALID_ARG;
+  if (N > (int64_t{1} << 40) / K) return BL_ERR_UNSUPPORTED;
+  if (!aligned(W, 4) || !aligned(buckets, 8)) return BL_ERR_ALIGNMENT;
+  int sms = 148;
+  bl_status st = device_info(&sms);
+  if (st != BL_OK) return st;
+  const cudaStream_t s = as_stream(stream);
+  auto* b = static_cast<unsigned long long*>(buckets);
+  bl::k_zero_u64<<<1, 256, 0, s>>>(b, bl::kBuckets);
+  if ((st = launch_status()) != BL_OK) return st;
+  const int64_t count = N * K;
+  int64_t ctas = (count / 4 + 255) / 256;
+  if (ctas > static_cast<int64_t>(sms) * 8) ctas = static_cast<int64_t>(sms) * 8;
+  if (ctas < 1) ctas = 1;
+  bl::k_absmean_buckets<<<static_cast<int>(ctas), 256, 0, s>>>(W, count, b);
+  return launch_status();
+}
+
+bl_status bitlinear_gamma_from_buckets(const void* buckets, int64_t count, float* gamma,
+                                       void* stream) {
+  if (!buckets || !gamma || count < 1) return BL_ERR_INVALID_ARG;
+  if (count > (int64_t{1} << 40)) return BL_ERR_UNSUPPORTED;  // bucket totals stay below 2^64
+  if (!aligned(buckets, 8) || !aligned(gamma, 4)) return BL_ERR_ALIGNMENT;
+  int sms = 148;
+  const bl_status st = device_info(&sms);
+  if (st != BL_OK) return st;
+  bl::k_gamma_finalize<<<1, 32, 0, as_stream(stream)>>>(
+      static_cast<const unsigned long long*>(buckets), count, gamma);
+  return launch_status();
+}
+
+bl_status bitlinear_ternarise_pack(const float* W, int64_t N, int64_t K, const float* gamma,
+                                   uint8_t* packed, void* stream) {
+  if (!W || !gamma || !packed) return BL_ERR_INVALID_ARG;
+  if (N < 1 || K < 1) return BL_ERR_INVALID_ARG;
+  if (N > (int64_t{1} << 40) / K) return BL_ERR_UNSUPPORTED;
+  if (!aligned(W, 4) || !aligned(gamma, 4)) return BL_ERR_ALIGNMENT;
+  int sms = 148;
+  const bl_status st = device_info(&sms);
+  if (st != BL_OK) return st;
+  const int64_t bytes = N * ((K + 3) / 4);
+  int64_t pctas = (bytes + 255) / 256;
+  if (pctas > static_cast<int64_t>(sms) * 32) pctas = static_cast<int64_t>(sms) * 32;
+  bl::k_ternarise_pack2<<<static_cast<int>(pctas), 256, 0, as_stream(stream)>>>(W, N, K, gamma,
+                                                                                packed);
+  return launch_status();
+}
+
 bl_status bitlinear_pack_weights(const float* W, int64_t N, int64_t K, uint8_t* packed,
                                  float* gamma, void* workspace, void* stream) {
   if (!W || !packed || !gamma || !workspace) return BL_ERR_INVALID_ARG;
   if (N < 1 || K < 1) return BL_ERR_INVALID_ARG;
   if (N > (int64_t{1} << 40) / K) return BL_ERR_UNSUPPORTED;
   if (!aligned(W, 4) || !aligned(workspace, 8) || !aligned(gamma, 4)) return BL_ERR_ALIGNMENT;
-  int sms = 148;
-  bl_status st = device_info(&sms);
+  bl_status st = bitlinear_absmean_buckets(W, N, K, workspace, stream);
   if (st != BL_OK) return st;
-  const cudaStream_t s = as_stream(stream);
-  auto* buckets = static_cast<unsigned long long*>(workspace);
-  bl::k_zero_u64<<<1, 256, 0, s>>>(buckets, bl::kBuckets);
-  if ((st = launch_status()) != BL_OK) return st;
-  const int64_t count = N * K;
-  int64_t ctas = (count / 4 + 255) / 256;
-  if (ctas > static_cast<int64_t>(sms) * 8) ctas = static_cast<int64_t>(sms) * 8;
-  if (ctas < 1) ctas = 1;
-  bl::k_absmean_buckets<<<static_cast<int>(ctas), 256, 0, s>>>(W, count, buckets);
-  if ((st = launch_status()) != BL_OK) return st;
-  bl::k_gamma_finalize<<<1, 32, 0, s>>>(buckets, count, gamma);
-  if ((st = launch_status()) != BL_OK) return st;
-  const int64_t bytes = N * ((K + 3) / 4);
-  int64_t pctas = (bytes + 255) / 256;
-  if (pctas > static_cast<int64_t>(sms) * 32) pctas = static_cast<int64_t>(sms) * 32;
-  bl::k_ternarise_pack2<<<static_cast<int>(pctas), 256, 0, s>>>(W, N, K, gamma, packed);
-  return launch_status();
+  if ((st = bitlinear_gamma_from_buckets(workspace, N * K, gamma, stream)) != BL_OK) return st;
+  return bitlinear_ternarise_pack(W, N, K, gamma, packed, stream);
 }
 
 bl_status bitlinear_rmsnorm_quant_act(const void* x, bl_dtype xdt, int64_t M, int64_t K,

@@ -61,6 +61,19 @@ def test_bad_arguments_are_rejected_without_a_launch(L):
     assert L.bitlinear_quant_act(fake, 0, 1, 0, fake, fake, fake, None) == _lib.BL_ERR_INVALID_ARG
     assert L.bitlinear_quant_act(P(257), 1, 1, 4, fake, fake, fake, None) == _lib.BL_ERR_ALIGNMENT
     assert L.bitlinear_quant_act(fake, 0, 0, 4, fake, fake, fake, None) == _lib.BL_OK  # M = 0: no-op
+    ab, gb, tp = L.bitlinear_absmean_buckets, L.bitlinear_gamma_from_buckets, L.bitlinear_ternarise_pack
+    assert ab(None, 4, 4, fake, None) == _lib.BL_ERR_INVALID_ARG
+    assert ab(fake, 0, 4, fake, None) == _lib.BL_ERR_INVALID_ARG
+    assert ab(fake, 1 << 21, 1 << 20, fake, None) == _lib.BL_ERR_UNSUPPORTED
+    assert ab(fake, 4, 4, P(260), None) == _lib.BL_ERR_ALIGNMENT
+    assert gb(None, 16, fake, None) == _lib.BL_ERR_INVALID_ARG
+    assert gb(fake, 0, fake, None) == _lib.BL_ERR_INVALID_ARG
+    assert gb(fake, (1 << 40) + 1, fake, None) == _lib.BL_ERR_UNSUPPORTED
+    assert gb(P(260), 16, fake, None) == _lib.BL_ERR_ALIGNMENT
+    assert tp(fake, 4, 4, None, fake, None) == _lib.BL_ERR_INVALID_ARG
+    assert tp(fake, 4, -1, fake, fake, None) == _lib.BL_ERR_INVALID_ARG
+    assert tp(fake, 1 << 21, 1 << 20, fake, fake, None) == _lib.BL_ERR_UNSUPPORTED
+    assert tp(P(258), 4, 4, fake, fake, None) == _lib.BL_ERR_ALIGNMENT
     rq = L.bitlinear_rmsnorm_quant_act
     assert rq(None, 1, 1, 4, fake, fake, fake, None) == _lib.BL_ERR_INVALID_ARG
     assert rq(None, 1, 0, 4, None, None, None, None) == _lib.BL_OK
