@@ -25,6 +25,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -94,10 +95,11 @@ CLOCK_Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active
 
 
 class ClockSampler:
-    def __init__(self, gpu_index):
+    def __init__(self, gpu_index, log_dir=None):
         self.gpu = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", "clocks_bench_%d.csv" % os.getpid())
+        self.path = os.path.join(log_dir or tempfile.gettempdir(),
+                                 "clocks_bench_%d.csv" % os.getpid())
 
     def __enter__(self):
         try:
@@ -261,7 +263,7 @@ def run_ours(args, world, rank, local):
         if g_rem:
             g_rem.replay()
 
-    with ClockSampler(local) as clk:
+    with ClockSampler(local, args.clocks_dir) as clk:
         t_step = timed(replays, stream, world)
         if t_step < 1.0:  # keep the clock sampler's window long enough
             pass
@@ -523,7 +525,7 @@ def make_bench_mats(wl_name, M, dev, stream, l2, copies=None):
 
 
 def run_sweep(mats, stream, world, peaks, Ms=(4, 8, 16, 32, 64)):
-    """decode_3b at the other batch sizes SURVEY-style: GB/s against HBM."""
+    """decode_3b at the other batch sizes: GB/s against HBM."""
     from ternary_weight_linear_04_b200 import bitlinear as bl
     hbm = float(peaks["hbm_gbs"])
     rows = []
@@ -856,6 +858,8 @@ def main():
                     help="comma list of extra sections: e2e,prefill,pack,sweep,layer70b,crossover,base3,"
                          "rmsnorm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--clocks-dir", default=None,
+                    help="folder for the raw nvidia-smi clock samples (default: the temp folder)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-seconds", type=float, default=120.0,
                     help="--impl reference: total CPU time of warm-up + timed steps")

@@ -22,7 +22,7 @@ Citations (page title tags as in ``bitlinear_oracle.c``):
                                BitLinear158.forward (rsqrt(mean(x^2) + 1e-6))
   base-3 packing            -- [Additive] "Energy, Memory Bandwidth, and
                                Serving Economics" (compact ternary packing,
-                               named only: the layout is this build's
+                               named only: the layout is this library's
                                reading, see pack3)
   rescale                   -- [Production] pipeline figure step 5,
                                BitLinear158.forward
@@ -91,7 +91,7 @@ def unpack2(packed, K):
 
 def packed3_stride(K):
     """Row stride of the base-3 layout: ceil(K/5) bytes rounded up to a
-    multiple of 16 (this build's reading; the pages give no layout)."""
+    multiple of 16 (this library's reading; the pages give no layout)."""
     return 16 * ((((K + 4) // 5) + 15) // 16)
 
 

@@ -1,9 +1,8 @@
 """bench.py's multi-rank plumbing on CPU: two gloo ranks on 127.0.0.1.
 
-The GPU runs of this build have one GPU, so the N > 1 path of bench.py
-(one process per GPU, max over ranks of the timed region, rank 0 alone
-prints; the reference arm runs on rank 0 only) is covered here with the
-gloo backend and no GPU.
+The N > 1 path of bench.py (one process per GPU, max over ranks of the
+timed region, rank 0 alone prints; the reference arm runs on rank 0 only)
+is covered here with the gloo backend and no GPU.
 """
 import json
 import os
@@ -57,7 +56,7 @@ def test_max_over_ranks_and_barrier_on_two_gloo_ranks():
 
 
 def test_reference_arm_under_torchrun_prints_once_on_rank_0():
-    """`--impl reference` launched like the driver's N=2 run: rank 0 times the
+    """`--impl reference` launched as a two-GPU run is (torchrun, two ranks): rank 0 times the
     CPU oracle and prints one JSON line; rank 1 exits 0 without work."""
     port = _free_port()
     cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
