@@ -765,7 +765,8 @@ def run_pack(mats, stream, world):
 
 def run_cpu_baseline(seconds):
     """The CPU oracle (scalar C, OpenMP over output rows) on the same
-    workload, as it stands, for about `seconds` seconds."""
+    workload, as it stands: about `seconds` seconds on every host thread,
+    then about a third of that on one thread."""
     from oracle import native as orc
     from ternary_weight_linear_04_b200 import inputs
     wl = inputs.WORKLOADS[WORKLOAD]
@@ -774,22 +775,28 @@ def run_cpu_baseline(seconds):
         W, x = inputs.make_matrix_inputs(wl, j, m_max=1)
         packed, gamma, _ = orc.pack_weights(W)
         mats.append((W.shape[1], W.shape[0], x, packed, gamma))
-    threads = orc.max_threads()
-    steps = 0
-    t0 = time.perf_counter()
-    while True:
-        for K, N, x, packed, gamma in mats:
-            xq, eta, _ = orc.quant_act(x)
-            orc.forward(xq, eta, packed, gamma, K, N, want_y_int=False)
-        steps += 1
-        if time.perf_counter() - t0 >= seconds:
-            break
-    t = time.perf_counter() - t0
     b = sum(linear_bytes(1, K, N) for K, N, *_ in mats)
+
+    def timed_steps(budget, nthreads):
+        steps = 0
+        t0 = time.perf_counter()
+        while True:
+            for K, N, x, packed, gamma in mats:
+                xq, eta, _ = orc.quant_act(x)
+                orc.forward(xq, eta, packed, gamma, K, N, nthreads=nthreads, want_y_int=False)
+            steps += 1
+            if time.perf_counter() - t0 >= budget:
+                return steps, time.perf_counter() - t0
+
+    threads = orc.max_threads()
+    steps, t = timed_steps(seconds, 0)
+    steps1, t1 = timed_steps(seconds / 3.0, 1)
     return {"value": round(b * steps / t / 1e9, 4), "unit": "GB/s", "cores": threads,
             "kind": "oracle",
             "sample": "%d full decode_3b steps (M=1, both matrices) in %.1f s on %d host threads"
-                      % (steps, t, threads)}
+                      % (steps, t, threads),
+            "single_thread": {"value": round(b * steps1 / t1 / 1e9, 4), "unit": "GB/s",
+                              "sample": "%d steps in %.1f s on 1 thread" % (steps1, t1)}}
 
 
 # ----------------------------------------------------------------- reference arm
