@@ -295,17 +295,24 @@ class BitLinear:
 
     ``BitLinear.from_latent(W)`` packs fp32 latent weights (N x K) once;
     calling the object quantises x (M x K) per token and runs the integer
-    accumulate + rescale."""
+    accumulate + rescale.  With ``rmsnorm=True`` the tokens are first
+    RMS-normalised (no affine weight, eps 1e-6; bf16 x), as BitLinear158.forward
+    does in [Production] "2. Absmax Dynamic Activation Quantization"."""
 
-    def __init__(self, packed, gamma, in_features, out_features):
+    def __init__(self, packed, gamma, in_features, out_features, rmsnorm=False):
         self.packed, self.gamma = packed, gamma
         self.in_features, self.out_features = in_features, out_features
+        self.rmsnorm = rmsnorm
 
     @classmethod
-    def from_latent(cls, W, stream=None):
+    def from_latent(cls, W, stream=None, rmsnorm=False):
         packed, gamma = pack_weights(W, stream=stream)
-        return cls(packed, gamma, W.shape[1], W.shape[0])
+        return cls(packed, gamma, W.shape[1], W.shape[0], rmsnorm=rmsnorm)
 
     def __call__(self, x, out_dtype=torch.bfloat16, stream=None):
+        if self.rmsnorm:
+            xq, eta, xsum = rmsnorm_quant_act(x, stream=stream)
+            return forward(xq, eta, xsum, self.packed, self.gamma, self.out_features,
+                           out_dtype=out_dtype, stream=stream, weights_static=True)
         return linear(x, self.packed, self.gamma, self.out_features, out_dtype=out_dtype,
                       weights_static=True, stream=stream)

@@ -101,3 +101,20 @@ def test_rmsnorm_then_layer_decode_3b(idx):
                               out_dtype=torch.float32, want_int=True)
         np.testing.assert_array_equal(y_int.cpu().numpy(), ref_yint[:M])
         np.testing.assert_array_equal(y.cpu().numpy().view(np.uint32), ref_y[:M].view(np.uint32))
+
+
+def test_bitlinear_module_with_rmsnorm():
+    """BitLinear(rmsnorm=True): norm, quantise, accumulate, rescale, against
+    the oracle's chain on the same inputs (fp32 and bf16 outputs)."""
+    N, K = 200, 512
+    W, x = inputs.make_case(4600, 3, K, N, act_dtype="bf16")
+    layer = bl.BitLinear.from_latent(torch.from_numpy(W).cuda(), rmsnorm=True)
+    xd = torch.from_numpy(x).cuda().to(torch.bfloat16)
+    ref_packed, ref_gamma, _ = orc.pack_weights(W)
+    want_q, want_eta, _ = ref.rmsnorm_quant_act(x)
+    _, ref_y = orc.forward(want_q, want_eta, ref_packed, ref_gamma, K, N)
+    y = layer(xd, out_dtype=torch.float32)
+    np.testing.assert_array_equal(y.cpu().numpy().view(np.uint32), ref_y.view(np.uint32))
+    yb = layer(xd)
+    np.testing.assert_array_equal(yb.cpu().view(torch.int16).numpy().view(np.uint16),
+                                  orc.f32_to_bf16_bits(ref_y))
