@@ -5,7 +5,6 @@ TEST INFRASTRUCTURE ONLY (see ``oracle/__init__.py``).  Same definitions as
 for the NumPy twin and for the timed CPU baseline.
 """
 import ctypes
-import os
 
 import numpy as np
 

@@ -17,8 +17,8 @@ decoder projections): W ~ N(0, 0.02^2) or Laplace(0, 0.02); x ~ N(0, 1) or
 Student-t(3) with 1% of channels scaled by 50 (an outlier stress case).
 """
 import math
-from dataclasses import dataclass, field
-from typing import List, Tuple
+from dataclasses import dataclass
+from typing import Tuple
 
 import numpy as np
 
