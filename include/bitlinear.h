@@ -275,7 +275,9 @@ bl_status bitlinear_forward_path(const int8_t* xq, const float* eta, const int32
  * ([Production] "2. Absmax Dynamic Activation Quantization"), accumulate
  * with add / subtract / skip ([Production] "The MatMul-Free Breakthrough")
  * and rescale ([Production] pipeline step 5).  Same results, bit for bit, as
- * bitlinear_quant_act followed by bitlinear_forward.
+ * bitlinear_quant_act followed by bitlinear_forward.  x is quantised as
+ * given; for the pages' BitLinear158 layer, which RMS-normalises first, call
+ * bitlinear_rmsnorm_quant_act and then bitlinear_forward.
  *
  *   x, xdt, M, K      in   activations as for bitlinear_quant_act.
  *   packed, gamma, N  in   as for bitlinear_forward.
