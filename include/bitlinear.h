@@ -87,7 +87,7 @@ size_t bitlinear_pack_workspace_bytes(void);
  * Implementation: The Lookup Table Approach".
  *
  *   W         in   fp32, N x K row-major (leading dimension K).
- *   N, K      in   out_features >= 1, in_features >= 1, N*K < 2^40.
+ *   N, K      in   out_features >= 1, in_features >= 1, N*K <= 2^40.
  *   packed    out  uint8, N x P with P = ceil(K/4) (bitlinear_packed_bytes):
  *                  byte n*P + k/4 holds code (W~[n,k] + 1) in bits
  *                  2*(k%4)..2*(k%4)+1, i.e. 00 = -1, 01 = 0, 10 = +1.
@@ -99,7 +99,7 @@ size_t bitlinear_pack_workspace_bytes(void);
  *                  overwritten; must not be shared by calls that may
  *                  overlap on the GPU.
  * Errors: BL_ERR_INVALID_ARG for null pointers or N, K < 1;
- * BL_ERR_UNSUPPORTED for N*K >= 2^40; BL_ERR_ALIGNMENT if workspace is not
+ * BL_ERR_UNSUPPORTED for N*K > 2^40; BL_ERR_ALIGNMENT if workspace is not
  * 8-byte or W not 4-byte aligned.
  */
 bl_status bitlinear_pack_weights(const float* W, int64_t N, int64_t K,
@@ -129,7 +129,7 @@ bl_status bitlinear_pack_weights(const float* W, int64_t N, int64_t K,
  */
 
 /* Step 1: zero `buckets`, then add the shard's |W| (fp32, N x K row-major,
- * N*K < 2^40).  Errors as bitlinear_pack_weights (buckets in place of
+ * N*K <= 2^40).  Errors as bitlinear_pack_weights (buckets in place of
  * workspace). */
 bl_status bitlinear_absmean_buckets(const float* W, int64_t N, int64_t K, void* buckets,
                                     void* stream);
@@ -145,7 +145,7 @@ bl_status bitlinear_gamma_from_buckets(const void* buckets, int64_t count, float
 /* Step 3: ternarise rows of W (N x K) with the given device gamma and pack
  * them as bitlinear_pack_weights does (N x ceil(K/4) bytes).  Errors:
  * BL_ERR_INVALID_ARG for null pointers or N, K < 1; BL_ERR_UNSUPPORTED for
- * N*K >= 2^40; BL_ERR_ALIGNMENT if W or gamma is not 4-byte aligned. */
+ * N*K > 2^40; BL_ERR_ALIGNMENT if W or gamma is not 4-byte aligned. */
 bl_status bitlinear_ternarise_pack(const float* W, int64_t N, int64_t K, const float* gamma,
                                    uint8_t* packed, void* stream);
 
@@ -162,7 +162,7 @@ bl_status bitlinear_ternarise_pack(const float* W, int64_t N, int64_t K, const f
  * the library (256 x 64-bit), held on every GPU that loads the library until
  * the process exits.  The call allocates nothing (no cudaMalloc, cudaFree
  * or allocating library routine).
- *   - Limit: N*K < 2^40 (the exact sum's 64-bit buckets); larger sizes return
+ *   - Limit: N*K <= 2^40 (the exact sum's 64-bit buckets); larger sizes return
  *     BL_ERR_UNSUPPORTED before anything is launched.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress, with that device current) and caches it; make

@@ -29,23 +29,33 @@ def sources():
                   + [os.path.join(INCLUDE, "bitlinear.h")])
 
 
-def needs_build():
-    if not os.path.exists(LIB):
+# The fault-injection variant used only by the timeout test: the same
+# sources with BL_TEST_HOOKS (1 ms wait limit, bitlinear_test_set_fault).
+TEST_HOOKS_LIB = os.path.join(HERE, "libbitlinear_testhooks.so")
+
+
+def needs_build(lib=LIB):
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return any(os.path.getmtime(s) > t for s in sources())
 
 
-def build(force=False, verbose=False, extra=()):
-    if not force and not needs_build():
-        return LIB
-    tmp = LIB + ".tmp%d" % os.getpid()
+def build(force=False, verbose=False, extra=(), lib=LIB):
+    if not force and not needs_build(lib):
+        return lib
+    tmp = lib + ".tmp%d" % os.getpid()
     cmd = [NVCC, *FLAGS, *extra, "-I", INCLUDE, os.path.join(CSRC, "bitlinear.cu"), "-o", tmp]
     if verbose:
         print(" ".join(cmd))
     subprocess.check_call(cmd)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
+
+
+def build_test_hooks(force=False):
+    """Builds the fault-injection variant (tests only; never loaded by the package)."""
+    return build(force=force, extra=("-DBL_TEST_HOOKS",), lib=TEST_HOOKS_LIB)
 
 
 if __name__ == "__main__":

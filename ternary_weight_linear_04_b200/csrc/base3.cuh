@@ -25,6 +25,19 @@ namespace bl {
 constexpr int kG3Warps = 8;
 constexpr int kG3Rows = 4;
 
+// Arguments of one k_gemv3 launch (MT tokens starting at xq).
+struct G3Launch {
+  const int8_t* xq;
+  const float* eta;
+  const int32_t* xsum;
+  int M, K, S;
+  const uint8_t* packed3;
+  const float* gamma;
+  int N;
+  void* y;
+  int32_t* y_int;
+};
+
 __device__ __forceinline__ uint4 ld_nc_v4(const uint8_t* p) {
   uint4 v;
   asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"

@@ -412,6 +412,23 @@ bl_status launch_generic(const int8_t* xq, const float* eta, int64_t M, int64_t 
   return BL_OK;
 }
 
+// Base-3 accumulate: shared memory of one launch (table, activation slots
+// of mt tokens, per-token scale and sum), and the launch itself.  The
+// attribute cache is per kernel instantiation (each k_gemv3<MT, OutT> has
+// its own static flags), so every instantiation gets its own raised
+// shared-memory limit and carveout.
+inline int64_t g3_smem(int mt, int64_t S) { return 2048 + static_cast<int64_t>(mt) * S * 8 + 64; }
+
+template <int MT, typename OutT>
+bl_status launch_gemv3(const bl::G3Launch& L, unsigned grid, cudaStream_t st) {
+  static int done[kMaxDevices] = {0};
+  auto kern = bl::k_gemv3<MT, OutT>;
+  const size_t smem = static_cast<size_t>(g3_smem(MT, L.S));
+  if (!ensure_smem(kern, smem, done)) return BL_ERR_CUDA;
+  return launch_pdl(kern, dim3(grid), dim3(32 * bl::kG3Warps), smem, st, L.xq, L.eta, L.xsum, L.M,
+                    L.K, L.S, L.packed3, L.gamma, L.N, L.y, L.y_int);
+}
+
 // K split of the tensor-core kernel: when the output tiles cannot fill the
 // GPU (few tokens), CTAs split K in clusters of up to 8 and add their
 // partial tiles in distributed shared memory.  floor(SMs / tiles) splits
@@ -770,11 +787,11 @@ bl_status bitlinear_forward3(const int8_t* xq, const float* eta, const int32_t* 
   if (M == 0) return BL_OK;
   if (!xq || !eta || !xsum || !y) return BL_ERR_INVALID_ARG;
   const int64_t S = bitlinear_packed3_stride(K);
-  // shared memory: the 2 KB table + 8-byte activation slots per group of five
-  // per token, kept within the 48 KB default (tokens per launch 4, 2 or 1)
-  constexpr int64_t kSmemLimit = 48 * 1024;
-  if (K > (1 << 30) || N > INT32_MAX / 2 || 2048 + S * 8 + 64 > kSmemLimit) return BL_ERR_UNSUPPORTED;
-  const int mt_max = 2048 + 4 * S * 8 + 64 <= kSmemLimit ? 4 : (2048 + 2 * S * 8 + 64 <= kSmemLimit ? 2 : 1);
+  // shared memory: the 2 KB table + 8-byte activation slots per group of
+  // five per token; tokens per launch 4, 2 or 1, the most that fit
+  const int64_t limit = static_cast<int64_t>(kDecMaxSmem);
+  if (K > (1 << 30) || N > INT32_MAX / 2 || g3_smem(1, S) > limit) return BL_ERR_UNSUPPORTED;
+  const int mt_max = g3_smem(4, S) <= limit ? 4 : (g3_smem(2, S) <= limit ? 2 : 1);
   if (!aligned(packed3, 16) || !aligned(eta, 4) || !aligned(xsum, 4) || !aligned(gamma, 4) ||
       (y_int && !aligned(y_int, 4)) || !aligned(y, ydt == BL_F32 ? 4 : 2))
     return BL_ERR_ALIGNMENT;
@@ -788,22 +805,19 @@ bl_status bitlinear_forward3(const int8_t* xq, const float* eta, const int32_t* 
   for (int64_t m0 = 0; m0 < M; m0 += mt_max) {
     const int mc = static_cast<int>(M - m0 < mt_max ? M - m0 : mt_max);
     const int mt = mc <= 1 ? 1 : (mc <= 2 ? 2 : 4);
-    const size_t smem = 2048 + static_cast<size_t>(mt) * S * 8 + 64;
     const int8_t* xq_m = xq + m0 * K;
     void* y_m = static_cast<char*>(y) + m0 * N * esz;
     int32_t* yi_m = y_int ? y_int + m0 * N : nullptr;
-    auto go = [&](auto kern) -> bl_status {
-      static int done[kMaxDevices] = {0};
-      if (!ensure_smem(kern, 0, done)) return BL_ERR_CUDA;  // carveout only: smem <= 48 KB
-      return launch_pdl(kern, dim3(static_cast<unsigned>(ctas)), dim3(32 * bl::kG3Warps), smem, cs,
-                        xq_m, eta + m0, xsum + m0, mc, static_cast<int>(K), static_cast<int>(S),
-                        packed3, gamma, static_cast<int>(N), y_m, yi_m);
-    };
+    const bl::G3Launch L = {xq_m, eta + m0, xsum + m0, mc, static_cast<int>(K), static_cast<int>(S),
+                            packed3, gamma, static_cast<int>(N), y_m, yi_m};
+    const unsigned grid = static_cast<unsigned>(ctas);
     if (ydt == BL_F32)
-      st = mt == 1 ? go(bl::k_gemv3<1, float>) : (mt == 2 ? go(bl::k_gemv3<2, float>) : go(bl::k_gemv3<4, float>));
+      st = mt == 1 ? launch_gemv3<1, float>(L, grid, cs)
+                   : (mt == 2 ? launch_gemv3<2, float>(L, grid, cs) : launch_gemv3<4, float>(L, grid, cs));
     else
-      st = mt == 1 ? go(bl::k_gemv3<1, __nv_bfloat16>)
-                   : (mt == 2 ? go(bl::k_gemv3<2, __nv_bfloat16>) : go(bl::k_gemv3<4, __nv_bfloat16>));
+      st = mt == 1 ? launch_gemv3<1, __nv_bfloat16>(L, grid, cs)
+                   : (mt == 2 ? launch_gemv3<2, __nv_bfloat16>(L, grid, cs)
+                              : launch_gemv3<4, __nv_bfloat16>(L, grid, cs));
     if (st != BL_OK) return st;
   }
   return BL_OK;
@@ -851,7 +865,7 @@ bl_status bitlinear_pack_weights_noalloc(const float* W, int64_t N, int64_t K, u
   if (!W || !packed || !gamma) return BL_ERR_INVALID_ARG;
   if (N < 1 || K < 1) return BL_ERR_INVALID_ARG;
   // The fixed 2048-byte scratch holds 64-bit bucket sums of 24-bit
-  // mantissas: exact for fewer than 2^40 weights.
+  // mantissas: exact for up to 2^40 weights.
   if (N > (int64_t{1} << 40) / K) return BL_ERR_UNSUPPORTED;
   if (!aligned(W, 4) || !aligned(gamma, 4)) return BL_ERR_ALIGNMENT;
   int sms = 148;
@@ -964,6 +978,17 @@ bl_path bitlinear_select_path(int64_t M, int64_t K, int64_t N, const void* xq, c
   (void)N;
   return select_path(M, K, xq, packed, y, y_int);
 }
+
+#ifdef BL_TEST_HOOKS
+// Fault-injection build only (not part of the library's interface): 1 makes
+// the tensor-core kernel withhold one barrier arrival, so that its bounded
+// wait runs out and the kernel returns with BL_ERR_TIMEOUT recorded; 0 turns
+// it off.  Synchronous.
+bl_status bitlinear_test_set_fault(int what) {
+  if (cudaMemcpyToSymbol(bl::g_test_fault, &what, sizeof(int)) != cudaSuccess) return BL_ERR_CUDA;
+  return cudaDeviceSynchronize() == cudaSuccess ? BL_OK : BL_ERR_CUDA;
+}
+#endif
 
 bl_status bitlinear_device_error(int32_t* code, void* stream) {
   if (!code) return BL_ERR_INVALID_ARG;

@@ -18,7 +18,15 @@ namespace bl {
 // reads and clears it.
 __device__ int g_device_error;
 
+#ifdef BL_TEST_HOOKS
+// Fault-injection build used only by the timeout test: waits give up after
+// 1 ms, and g_test_fault (set by bitlinear_test_set_fault) makes a kernel
+// withhold one barrier arrival so that a wait runs out.
+constexpr unsigned long long kWaitLimitNs = 1000000ull;  // 1 ms per wait
+__device__ int g_test_fault;
+#else
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s per wait
+#endif
 
 __device__ __forceinline__ unsigned long long globaltimer_ns() {
   unsigned long long t;
@@ -80,6 +88,19 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
       return false;
     }
   }
+}
+
+// After an abort: wait for a phase that an asynchronous copy or a tensor-core
+// commit already issued by this CTA will complete, so that nothing is still
+// writing into this CTA's shared memory (or reading its TMEM) when it exits.
+// Ignores the abort flag; bounded by kWaitLimitNs like every other wait.
+__device__ __forceinline__ bool mbar_drain(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+  }
+  return true;
 }
 
 // ---------------------------------------------------------------- TMA

@@ -70,7 +70,7 @@ struct TcCfg {
           ? 8
           : 1 + static_cast<int>(kStageRegion / (static_cast<size_t>(kTcBN) * BM * 4));
   static constexpr int kTmemCols = BM < 32 ? 32 : BM;
-  static constexpr int kBarBytes = 8 * (4 * kStages + 1) + 16 + 8 * BM;
+  static constexpr int kBarBytes = 8 * (4 * kStages + 2) + 16 + 8 * BM;
   static constexpr size_t kSmem = 1024 + kStageRegion + kBarBytes;
   static_assert(kSmem <= 227 * 1024, "shared memory per CTA");
   static_assert(BM > 32 || kSmem <= 113 * 1024, "two CTAs per SM for the small token tiles");
@@ -96,7 +96,8 @@ __global__ void __launch_bounds__(kTcThreads, BM <= 32 ? 2 : 1)
   uint64_t* full_b = full_p + S;  // activation tile in
   uint64_t* empty = full_b + S;   // the MMA is done with the stage
   uint64_t* accum_full = empty + S;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum_full + 1);
+  uint64_t* drain = accum_full + 1;  // the MMAs issued before an abort are done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* s_scale = reinterpret_cast<float*>(tmem_slot + 4);
   int32_t* s_xsum = reinterpret_cast<int32_t*>(s_scale + BM);
@@ -124,6 +125,7 @@ __global__ void __launch_bounds__(kTcThreads, BM <= 32 ? 2 : 1)
       mbar_init(empty + s, 1);
     }
     mbar_init(accum_full, 1);
+    mbar_init(drain, 1);
     *abort_flag = 0;
     mbar_init_fence();
     tma_prefetch_desc(&tm_x);
@@ -150,6 +152,7 @@ __global__ void __launch_bounds__(kTcThreads, BM <= 32 ? 2 : 1)
   tc_fence_after();
   const uint32_t tmem_d = *tmem_slot;
   bool epi_ok = false;  // unpack warps: the accumulator is complete
+  int issued = 0;       // warp 0, lane 0 / 1: activation / packed-weight loads issued
 
   if (warp == 0) {
     // ---------------- TMA producers: lane 0 activations, lane 1 packed weights
@@ -159,13 +162,16 @@ __global__ void __launch_bounds__(kTcThreads, BM <= 32 ? 2 : 1)
         if (i >= S && !mbar_wait(empty + s, static_cast<uint32_t>(i / S - 1) & 1u, abort_flag)) break;
         mbar_arrive_expect_tx(full_b + s, Cfg::kBBytes);
         tma_load_2d(sB + s * Cfg::kBBytes, &tm_x, full_b + s, (kt0 + i) * kTcBK, m0);
+        issued = i + 1;
       }
     } else if (lane == 1) {
       if (!wstatic)
         for (int i = 0; i < p_first; ++i) issue_p(i);
+      issued = p_first;
       for (int i = S; i < nkt; ++i) {
         if (!mbar_wait(empty + i % S, static_cast<uint32_t>(i / S - 1) & 1u, abort_flag)) break;
         issue_p(i);
+        issued = i + 1;
       }
     }
   } else if (warp == 1) {
@@ -183,7 +189,13 @@ __global__ void __launch_bounds__(kTcThreads, BM <= 32 ? 2 : 1)
         const int s = i % S;
         const uint32_t par = static_cast<uint32_t>(i / S) & 1u;
         ok = mbar_wait(full_b + s, par, abort_flag) && mbar_wait(full_a + s, par, abort_flag);
-        if (!ok) break;
+        if (!ok) {
+          if (i > 0) {  // MMAs are in flight: let them finish before TMEM is freed
+            tc_commit(drain);
+            mbar_drain(drain, 0);
+          }
+          break;
+        }
         tc_fence_after();
         const uint64_t ad = a_desc0 + static_cast<uint64_t>(s * (Cfg::kABytes >> 4));
         const uint64_t bd = b_desc0 + static_cast<uint64_t>(s * (Cfg::kBBytes >> 4));
@@ -225,10 +237,25 @@ __global__ void __launch_bounds__(kTcThreads, BM <= 32 ? 2 : 1)
       }
       fence_proxy_async_smem();
       __syncwarp();
+#ifdef BL_TEST_HOOKS
+      if (g_test_fault == 1 && u == 0 && i == 0) continue;  // a wait that nothing completes
+#endif
       if (lane == 0) mbar_arrive(full_a + s);
     }
     if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait(accum_full, 0, abort_flag));
-    epi_ok = ok;
+    epi_ok = ok && __all_sync(0xFFFFFFFFu, *abort_flag == 0);
+  }
+
+  // Every role is done and the abort flag is final.  After an abort, the
+  // producers wait (bounded) for their last S loads, the only ones that can
+  // still be in flight, so no copy lands in shared memory that is reused
+  // below or freed at exit.
+  __syncwarp();
+  __syncthreads();
+  if (warp == 0 && lane < 2 && *abort_flag) {
+    uint64_t* bars = lane == 0 ? full_b : full_p;
+    for (int i = issued > S ? issued - S : 0; i < issued; ++i)
+      mbar_drain(bars + i % S, static_cast<uint32_t>(i / S) & 1u);
   }
 
   // ---------------- epilogue (warps 2..9): one TMEM lane = one output feature

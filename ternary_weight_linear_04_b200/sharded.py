@@ -61,6 +61,7 @@ class ShardedBitLinear:
             raise ValueError("rank %d holds %d rows; its shard is [%d, %d)"
                              % (self.rank, W_shard.shape[0], self.n0, self.n1))
         self.n_max = -(-N // self.world)
+        self._bufs = {}
         if self.n1 > self.n0:
             buckets = ops.absmean_buckets(W_shard, stream=stream)
         else:  # more ranks than rows: this rank contributes nothing
@@ -81,14 +82,31 @@ class ShardedBitLinear:
         return self.ops.linear(x, self.packed, self.gamma, n, out_dtype=out_dtype,
                                weights_static=True, stream=stream, out=out)
 
-    def forward(self, x, out_dtype=torch.bfloat16, stream=None):
+    def _staging(self, M, dtype, device):
+        """The send block and the gather buffer for M tokens of `dtype`,
+        allocated on the first call with that shape and reused after it."""
+        key = (M, dtype, device)
+        bufs = self._bufs.get(key)
+        if bufs is None:
+            send = torch.empty(M * self.n_max, dtype=dtype, device=device)
+            recv = torch.empty(self.world * M * self.n_max, dtype=dtype, device=device)
+            bufs = self._bufs[key] = (send, recv)
+        return bufs
+
+    def forward(self, x, out_dtype=torch.bfloat16, stream=None, out=None):
         """The whole output y (M x N) on every rank: local columns, then one
         all-gather of equal-sized (padded) per-rank blocks along N.  The layer
         writes its columns straight into the send block when they are
-        contiguous there (one token, or an even split)."""
+        contiguous there (one token, or an even split); with one token and an
+        even split the gather lands directly in y.  The send block and the
+        gather buffer are kept between calls (per token count and dtype), so
+        a call allocates nothing but y itself, and not that when `out` (a
+        contiguous M x N tensor) is given."""
         M = x.shape[0]
         n = self.n1 - self.n0
-        send = torch.empty(M * self.n_max, dtype=out_dtype, device=x.device)
+        if out is None:
+            out = torch.empty((M, self.N), dtype=out_dtype, device=x.device)
+        send, recv = self._staging(M, out_dtype, x.device)
         if n > 0 and (M == 1 or n == self.n_max):
             self.forward_local(x, out_dtype, stream, out=send[:M * n].view(M, n))
             _after(stream, x.device)
@@ -96,13 +114,14 @@ class ShardedBitLinear:
             y_local = self.forward_local(x, out_dtype, stream)
             _after(stream, x.device)
             send.view(M, self.n_max)[:, :n] = y_local
-        recv = torch.empty(self.world * M * self.n_max, dtype=out_dtype, device=x.device)
+        if self.n_max * self.world == self.N and M == 1 and out.is_contiguous():
+            # rank-major blocks are already y's layout
+            dist.all_gather_into_tensor(out.view(-1), send, group=self.group)
+            return out
         dist.all_gather_into_tensor(recv, send, group=self.group)
         blocks = recv.view(self.world, M, self.n_max)
-        if self.n_max * self.world == self.N and M == 1:
-            return blocks.view(1, self.N)  # rank-major blocks are already y's layout
         parts = []
         for r in range(self.world):
             a, b = shard_bounds(self.N, self.world, r)
             parts.append(blocks[r, :, :b - a])
-        return torch.cat(parts, dim=1)
+        return torch.cat(parts, dim=1, out=out)

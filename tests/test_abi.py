@@ -65,6 +65,7 @@ def test_bad_arguments_are_rejected_without_a_launch(L):
     assert ab(None, 4, 4, fake, None) == _lib.BL_ERR_INVALID_ARG
     assert ab(fake, 0, 4, fake, None) == _lib.BL_ERR_INVALID_ARG
     assert ab(fake, 1 << 21, 1 << 20, fake, None) == _lib.BL_ERR_UNSUPPORTED
+    assert ab(fake, (1 << 20) + 1, 1 << 20, fake, None) == _lib.BL_ERR_UNSUPPORTED  # one row past N*K = 2^40
     assert ab(fake, 4, 4, P(260), None) == _lib.BL_ERR_ALIGNMENT
     assert gb(None, 16, fake, None) == _lib.BL_ERR_INVALID_ARG
     assert gb(fake, 0, fake, None) == _lib.BL_ERR_INVALID_ARG

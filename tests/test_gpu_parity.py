@@ -573,3 +573,56 @@ def test_forward3_matches_the_oracle(M, K, N, out):
     y, y_int = bl.forward3(xq, eta, xsum, packed3, gamma, N, out_dtype=DT[out], want_int=True)
     np.testing.assert_array_equal(y_int.cpu().numpy(), ref_yint)
     np.testing.assert_array_equal(y_bits(y.cpu()), oracle_y_bits(ref_y, out))
+
+
+# ----------------------------------------------------------------- the headline decode call
+
+@pytest.mark.parametrize("M", [1, 2, 4, 16])
+def test_headline_decode_call_every_output(M):
+    """The call the decode benchmark times: bitlinear_linear on both decode_3b
+    matrices (K=3200 -> N=8640 and K=8640 -> N=3200) with static weights,
+    the benchmark's own seeded inputs, issued back to back on one stream with
+    no synchronisation between them (as the timed step does).  Every output
+    element, x~, eta, xsum and y_int are compared with the oracle bit for
+    bit ([Production] "The MatMul-Free Breakthrough" and pipeline step 5)."""
+    w = inputs.WORKLOADS["decode_3b"]
+    mats = []
+    for idx in range(2):
+        W, x = inputs.make_matrix_inputs(w, idx, m_max=max(M, 64))
+        ref_packed, ref_gamma, _ = orc.pack_weights(W)
+        _, _, packed, gamma = gpu_pack(W)
+        mats.append((W.shape, x[:M], ref_packed, ref_gamma, packed, gamma))
+    torch.cuda.synchronize()
+    outs = []
+    for (N, K), x, _, _, packed, gamma in mats:
+        xd = torch.from_numpy(x).cuda().to(torch.bfloat16)
+        outs.append(bl.linear(xd, packed, gamma, N, out_dtype=torch.bfloat16, want_quant=True,
+                              want_int=True, weights_static=True))
+    torch.cuda.synchronize()
+    for ((N, K), x, ref_packed, ref_gamma, _, _), (y, (xq, eta, xsum), y_int) in zip(mats, outs):
+        ref_xq, ref_eta, ref_xsum = orc.quant_act(x)
+        ref_yint, ref_y = orc.forward(ref_xq, ref_eta, ref_packed, ref_gamma, K, N)
+        np.testing.assert_array_equal(xq.cpu().numpy(), ref_xq)
+        np.testing.assert_array_equal(eta.cpu().numpy().view(np.uint32), ref_eta.view(np.uint32))
+        np.testing.assert_array_equal(xsum.cpu().numpy(), ref_xsum)
+        np.testing.assert_array_equal(y_int.cpu().numpy(), ref_yint)
+        np.testing.assert_array_equal(y_bits(y.cpu()), orc.f32_to_bf16_bits(ref_y))
+
+
+@pytest.mark.parametrize("M,K", [(4, 8192), (4, 28672), (3, 16384), (9, 8192)])
+def test_forward3_many_tokens_with_large_shared_memory(M, K):
+    """Base-3 launches whose activation slots need more than 48 KB of shared
+    memory (4 tokens at K = 8192 take 55 KB; at K = 28672 187 KB): each
+    kernel instantiation raises its own shared-memory limit, so these run as
+    four-token launches.  y_int and y bit-exact against the oracle."""
+    N = 515
+    W, x = inputs.make_case(9300 + M + K, M, K, N, act_dtype="bf16")
+    ref_packed, ref_gamma, _ = orc.pack_weights(W)
+    ref_xq, ref_eta, ref_xsum = orc.quant_act(x)
+    ref_yint, ref_y = orc.forward(ref_xq, ref_eta, ref_packed, ref_gamma, K, N)
+    packed3, gamma = bl.pack_weights3(torch.from_numpy(W).cuda())
+    xq, eta, xsum = (torch.from_numpy(a).cuda() for a in (ref_xq, ref_eta, ref_xsum))
+    for out in ("f32", "bf16"):
+        y, y_int = bl.forward3(xq, eta, xsum, packed3, gamma, N, out_dtype=DT[out], want_int=True)
+        np.testing.assert_array_equal(y_int.cpu().numpy(), ref_yint)
+        np.testing.assert_array_equal(y_bits(y.cpu()), oracle_y_bits(ref_y, out))
