@@ -270,6 +270,8 @@ def run_ours(args, world, rank, local):
     with ClockSampler(local, args.clocks_dir) as clk:
         t_first = max_over_ranks(timed(replays, stream, world), world)
         n_win = min(2000, max(5, int(np.ceil(0.05 / max(t_first, 1e-9)))))
+        if args.windows:
+            n_win = args.windows
         wins = [t_first] + [max_over_ranks(timed(replays, stream, world), world)
                             for _ in range(n_win - 1)]
     t_step = statistics.median(wins)
@@ -284,9 +286,14 @@ def run_ours(args, world, rank, local):
     achieved = bytes_per_launch / avg_launch / 1e9
     hbm_peak = float(peaks["hbm_gbs"])
     paths = [bl.select_path(M, m["K"], m["N"], m["xq"], m["copies"][0][0], m["y"]) for m in mats]
-    roofline = {"kernel": "k_decode (fused quantise + accumulate + rescale)",
+    # which fused decode kernel bitlinear_linear runs for each matrix
+    sms = props.multi_processor_count
+    reg_shapes = [bl.decode_reg_shape(m["K"], m["N"], sms) if M == 1 else None for m in mats]
+    kernel = "k_decode_reg" if all(reg_shapes) else "k_decode"
+    roofline = {"kernel": "%s (fused quantise + accumulate + rescale)" % kernel,
                 "bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
-                "frac": round(achieved / hbm_peak, 4), "traffic": load_traffic("k_decode"),
+                "frac": round(achieved / hbm_peak, 4), "traffic": load_traffic(kernel),
+                "shapes": reg_shapes if kernel == "k_decode_reg" else None,
                 "peak_source": peak_src + " hbm_gbs (burst copy)",
                 "avg_launch_us": round(avg_launch * 1e6, 3),
                 "algorithmic_bytes_per_launch": bytes_per_launch}
@@ -832,6 +839,56 @@ def run_cpu_baseline(seconds):
                               "sample": "%d steps in %.1f s on 1 thread" % (steps1, t1)}}
 
 
+# ----------------------------------------------------------------- profiling program
+
+def profile_kernels():
+    """Each kernel of the library, twice, at the size of the workload it
+    serves (for ncu: capture the second launch of a kernel with -s 1 -c 1,
+    or all of them): pack (decode_3b's 8640 x 3200 fp32 W), quantiser
+    (prefill_7b's 2048 x 4096), RMSNorm + quantiser (2048 x 8640), the
+    one-token decode kernels on both decode_3b matrices, the shared-memory
+    decode kernel at M = 4, the tensor-core kernel on prefill_7b, the base-3
+    kernel on decode_3b (K=3200 -> N=8640) and the generic kernel (M = 3,
+    K = 1000, N = 300)."""
+    from ternary_weight_linear_04_b200 import build as libbuild, inputs
+    from ternary_weight_linear_04_b200 import bitlinear as bl
+    libbuild.build()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    wl = inputs.WORKLOADS["decode_3b"]
+    mats = []
+    for j in range(2):
+        W, x = inputs.make_matrix_inputs(wl, j, m_max=4)
+        mats.append((torch.from_numpy(W).to(dev), torch.from_numpy(x).to(dev).to(torch.bfloat16)))
+    pw = inputs.WORKLOADS["prefill_7b"]
+    Wp, xp = inputs.make_matrix_inputs(pw, 0)
+    Wp = torch.from_numpy(Wp).to(dev)
+    xp = torch.from_numpy(xp).to(dev).to(torch.bfloat16)
+    rng = np.random.default_rng(5)
+    xr = torch.from_numpy(inputs.draw_activations(rng, 2048, 8640, "normal", "bf16")).to(dev).to(torch.bfloat16)
+    torch.cuda.synchronize()
+    for _ in range(2):
+        packed = [bl.pack_weights(W) for W, _ in mats]
+        bl.quant_act(xp)
+        bl.rmsnorm_quant_act(xr)
+        for (pk, g), (W, x) in zip(packed, mats):
+            bl.linear(x[:1], pk, g, W.shape[0], weights_static=True)
+        pk, g = packed[0]
+        bl.linear(mats[0][1][:4], pk, g, mats[0][0].shape[0], weights_static=True)
+        ppk, pg = bl.pack_weights(Wp)
+        xq, eta, xsum = bl.quant_act(xp)
+        bl.forward(xq, eta, xsum, ppk, pg, Wp.shape[0], weights_static=True)
+        p3, g3 = bl.pack_weights3(mats[0][0])
+        xq1, eta1, xsum1 = bl.quant_act(mats[0][1][:1])
+        bl.forward3(xq1, eta1, xsum1, p3, g3, mats[0][0].shape[0])
+        Wg, xg = inputs.make_case(77, 3, 1000, 300)
+        pkg, gg = bl.pack_weights(torch.from_numpy(Wg).to(dev))
+        xqg, etag, xsg = bl.quant_act(torch.from_numpy(xg).to(dev))
+        bl.forward(xqg, etag, xsg, pkg, gg, 300, path="generic")
+        torch.cuda.synchronize()
+    print(json.dumps({"profile_kernels": "done", "device": torch.cuda.get_device_name(dev)}))
+
+
 # ----------------------------------------------------------------- reference arm
 
 def run_reference(args, world, rank):
@@ -903,10 +960,18 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-seconds", type=float, default=120.0,
                     help="--impl reference: total CPU time of warm-up + timed steps")
+    ap.add_argument("--windows", type=int, default=0,
+                    help="number of timed windows of --steps steps (default: >= 5 and >= 50 ms)")
+    ap.add_argument("--profile-kernels", action="store_true",
+                    help="run each library kernel twice at its workload's size and exit "
+                         "(a short program for ncu captures; prints one line)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     world, rank, local = dist_setup(args.gpus)
+    if args.profile_kernels:
+        profile_kernels()
+        return
     try:
         if args.impl == "reference":
             out = run_reference(args, world, rank)

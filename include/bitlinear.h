@@ -287,7 +287,10 @@ bl_status bitlinear_forward_path(const int8_t* xq, const float* eta, const int32
  *                          two tokens (M <= 2, K % 64 == 0, K * M' <=
  *                          131072 with M' = M rounded up to 1 or 2, 16-byte
  *                          aligned x, packed, y) one fused kernel runs and
- *                          these are optional (NULL = not written).
+ *                          these are optional (NULL = not written).  For
+ *                          one token whose layer fits it (see
+ *                          bitlinear_decode_reg_shape), that kernel holds
+ *                          each CTA's weights in registers.
  *                          Otherwise two kernels run (quantiser, then the
  *                          accumulate kernel bitlinear_forward would pick)
  *                          and they are required scratch
@@ -325,11 +328,30 @@ bl_status bitlinear_decode_shape_for(int64_t M, int64_t K, int64_t N, int fused,
                                      int32_t* shape);
 
 /*
+ * Shape of the one-token fused kernel of bitlinear_linear that holds each
+ * CTA's weights in registers, for K inputs and N outputs on a GPU with `sms`
+ * SMs (host logic only; usable without a GPU).  The pages have no
+ * counterpart: this describes how the library lays the add / subtract /
+ * skip accumulation of one token out on the GPU.  bitlinear_linear uses this
+ * kernel for M = 1 (bf16 x, K % 64 == 0, the fused conditions above) when
+ * this query succeeds and no decode shape is forced
+ * (bitlinear_set_decode_shape); otherwise the shared-memory decode kernel.
+ * shape (host, 4 int32) receives: rows per warp RB (1, 2 or 4; 16 warps per
+ * CTA), 32-bit weight words per lane and row NJ (K <= 512 NJ), rows per CTA,
+ * CTAs.  Errors: BL_ERR_INVALID_ARG for shape == NULL, K < 1, N < 1 or
+ * sms < 1; BL_ERR_UNSUPPORTED when the kernel does not take (K, N): K not a
+ * multiple of 64, more than 64 rows per CTA, or more weight words than its
+ * register budget.
+ */
+bl_status bitlinear_decode_reg_shape(int64_t K, int64_t N, int sms, int32_t* shape);
+
+/*
  * Force the decode kernel's shape for every later launch in this process:
  * team_warps G in 1..16 and rows_per_block RB in {1, 2, 4, 8, 16} (RB * M'
  * <= 16 with M' = M rounded up to 1, 2 or 4); 0 for either leaves that
  * choice to the library (the default).  A forced shape that a launch cannot
- * use makes that launch return BL_ERR_UNSUPPORTED.  Results are identical
+ * use makes that launch return BL_ERR_UNSUPPORTED.  While a shape is forced,
+ * bitlinear_linear runs the shared-memory decode kernel for one token too.  Results are identical
  * for every shape; this exists to test and tune the shapes.  Not
  * synchronised with launches in flight on other host threads.
  * Errors: BL_ERR_INVALID_ARG for values outside those ranges.

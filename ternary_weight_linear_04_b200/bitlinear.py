@@ -173,6 +173,20 @@ def decode_shape(M, K, N, fused=True):
     return dict(zip(DECODE_SHAPE_FIELDS, list(buf)))
 
 
+def decode_reg_shape(K, N, sms=None):
+    """Shape of the one-token register-resident kernel of bitlinear_linear for
+    (K, N) as a dict, or None when that kernel does not take the layer.  sms
+    defaults to the current device's SM count."""
+    if sms is None:
+        sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    buf = (ctypes.c_int32 * 4)()
+    st = _lib.lib().bitlinear_decode_reg_shape(K, N, sms, buf)
+    if st == _lib.BL_ERR_UNSUPPORTED:
+        return None
+    check(st, "bitlinear_decode_reg_shape")
+    return dict(zip(("rows_per_warp", "words_per_lane", "rows_per_cta", "ctas"), list(buf)))
+
+
 def set_tc_split(k_split=0):
     """Force the K split (CTAs per cluster) of the tensor-core kernel for later
     launches in this process (0 = the library's choice)."""

@@ -18,6 +18,7 @@
 #include "bitlinear.h"
 #include "common.cuh"
 #include "decode.cuh"
+#include "decode_reg.cuh"
 #include "base3.cuh"
 #include "gemm_tc.cuh"
 #include "gemv.cuh"
@@ -390,6 +391,62 @@ bl_status launch_decode(const bl::DecodeArgs& a, int sms, cudaStream_t st) {
   }
 }
 
+// One-token layer with the CTA's weights in registers (decode_reg.cuh):
+// 16 warps of RB rows each, NJ 32-bit words per lane and row.  Applies when
+// one CTA per SM leaves at most 64 rows per CTA and the weight registers
+// (RB * NJ) stay within the 64-register budget; the instantiated word
+// counts cover the common layer widths (K <= 512 NJ, the smallest that fits
+// is taken; the unused words are predicated off).
+struct RegGeom {
+  int RB = 0, NJ = 0, rows_per_cta = 0, grid = 0;
+};
+
+constexpr int kRegNJ1[] = {2, 4, 7, 8, 12, 16, 17, 24};
+constexpr int kRegNJ2[] = {2, 4, 7, 8, 12, 16, 17};
+constexpr int kRegNJ4[] = {2, 4, 7, 8};
+
+bool reg_decode_geometry(int64_t K, int64_t N, int sms, RegGeom* g) {
+  if (K < 64 || K % 64 != 0 || N < 1 || N > INT32_MAX / 2) return false;
+  int64_t grid = N < sms ? N : sms;
+  const int64_t rpc = (N + grid - 1) / grid;
+  grid = (N + rpc - 1) / rpc;
+  const int RB = rpc <= 16 ? 1 : (rpc <= 32 ? 2 : (rpc <= 64 ? 4 : 0));
+  if (RB == 0) return false;
+  const int64_t need = (K / 16 + 31) / 32;
+  const int* list = RB == 1 ? kRegNJ1 : (RB == 2 ? kRegNJ2 : kRegNJ4);
+  const int n = RB == 1 ? 8 : (RB == 2 ? 7 : 4);
+  int NJ = 0;
+  for (int i = 0; i < n && !NJ; ++i)
+    if (list[i] >= need) NJ = list[i];
+  if (!NJ) return false;
+  g->RB = RB;
+  g->NJ = NJ;
+  g->rows_per_cta = static_cast<int>(rpc);
+  g->grid = static_cast<int>(grid);
+  return true;
+}
+
+template <int RB, int NJ>
+bl_status launch_decode_reg_nj(const bl::RegDecodeArgs& a, const RegGeom& g, cudaStream_t st) {
+  static int done[kMaxDevices] = {0};
+  auto kern = bl::k_decode_reg<RB, NJ>;
+  if (!ensure_smem(kern, 0, done)) return BL_ERR_CUDA;
+  return launch_pdl(kern, dim3(static_cast<unsigned>(g.grid)), dim3(bl::kRegThreads),
+                    static_cast<size_t>(32 * NJ * 16), st, a);
+}
+
+bl_status launch_decode_reg(const bl::RegDecodeArgs& a, const RegGeom& g, cudaStream_t st) {
+#define BL_REG_CASE(R, J) \
+  if (g.RB == R && g.NJ == J) return launch_decode_reg_nj<R, J>(a, g, st);
+  BL_REG_CASE(1, 2) BL_REG_CASE(1, 4) BL_REG_CASE(1, 7) BL_REG_CASE(1, 8) BL_REG_CASE(1, 12)
+  BL_REG_CASE(1, 16) BL_REG_CASE(1, 17) BL_REG_CASE(1, 24)
+  BL_REG_CASE(2, 2) BL_REG_CASE(2, 4) BL_REG_CASE(2, 7) BL_REG_CASE(2, 8) BL_REG_CASE(2, 12)
+  BL_REG_CASE(2, 16) BL_REG_CASE(2, 17)
+  BL_REG_CASE(4, 2) BL_REG_CASE(4, 4) BL_REG_CASE(4, 7) BL_REG_CASE(4, 8)
+#undef BL_REG_CASE
+  return BL_ERR_UNSUPPORTED;
+}
+
 template <typename OutT>
 bl_status launch_generic(const int8_t* xq, const float* eta, int64_t M, int64_t K,
                          const uint8_t* packed, const float* gamma, int64_t N, void* y,
@@ -635,6 +692,17 @@ bl_status bitlinear_decode_shape(int64_t M, int64_t K, int64_t N, int fused, int
   shape[7] = g.stages;
   shape[8] = g.x_staged;
   shape[9] = static_cast<int32_t>(g.smem);
+  return BL_OK;
+}
+
+bl_status bitlinear_decode_reg_shape(int64_t K, int64_t N, int sms, int32_t* shape) {
+  if (!shape || K < 1 || N < 1 || sms < 1) return BL_ERR_INVALID_ARG;
+  RegGeom g;
+  if (!reg_decode_geometry(K, N, sms, &g)) return BL_ERR_UNSUPPORTED;
+  shape[0] = g.RB;
+  shape[1] = g.NJ;
+  shape[2] = g.rows_per_cta;
+  shape[3] = g.grid;
   return BL_OK;
 }
 
@@ -963,12 +1031,33 @@ bl_status bitlinear_linear(const void* x, bl_dtype xdt, int64_t M, int64_t K, co
   int sms = 148;
   bl_status st = device_info(&sms);
   if (st != BL_OK) return st;
+  const cudaStream_t s = as_stream(stream);
+  // One token: the register-resident kernel when the CTA's share fits (and
+  // no decode shape is forced for the shared-memory kernel).
+  RegGeom rg;
+  if (M == 1 && g_force_G.load(std::memory_order_relaxed) == 0 &&
+      g_force_RB.load(std::memory_order_relaxed) == 0 && reg_decode_geometry(K, N, sms, &rg)) {
+    bl::RegDecodeArgs r = {};
+    r.x = static_cast<const __nv_bfloat16*>(x);
+    r.K = static_cast<int>(K);
+    r.N = static_cast<int>(N);
+    r.packed = packed;
+    r.gamma = gamma;
+    r.y = y;
+    r.y_bf16 = ydt == BL_BF16 ? 1 : 0;
+    r.y_int = y_int;
+    r.rows_per_cta = rg.rows_per_cta;
+    r.weights_static = (flags & BL_FLAG_WEIGHTS_STATIC) ? 1 : 0;
+    r.xq_out = xq;
+    r.eta_out = eta;
+    r.xsum_out = xsum;
+    return launch_decode_reg(r, rg, s);
+  }
   bl::DecodeArgs a = {};
   a.x = x; a.M = (int)M; a.K = (int)K; a.N = (int)N;
   a.packed = packed; a.gamma = gamma; a.y = y; a.y_int = y_int;
   a.weights_static = (flags & BL_FLAG_WEIGHTS_STATIC) ? 1 : 0;
   a.xq_out = xq; a.eta_out = eta; a.xsum_out = xsum;
-  const cudaStream_t s = as_stream(stream);
   return ydt == BL_F32 ? launch_decode<__nv_bfloat16, float>(a, sms, s)
                        : launch_decode<__nv_bfloat16, __nv_bfloat16>(a, sms, s);
 }

@@ -7,6 +7,7 @@
 // so a bug can never leave a GPU spinning forever.
 #pragma once
 
+#include <cmath>
 #include <cstdint>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
@@ -298,11 +299,28 @@ __device__ __forceinline__ void transpose4x4_bytes(uint32_t a0, uint32_t a1, uin
   o3 = __byte_perm(u2, u3, 0x7632);
 }
 
+// RN32(a / 127) without a divide: y = RN32(1/127), q0 = RN32(a y), the
+// remainder a - 127 q0 is exact (one fma), and RN32(q0 + (a - 127 q0) y) is
+// the correctly rounded quotient (P. Markstein, "IA-64 and Elementary
+// Functions", 2000: a faithful quotient corrected with the exact remainder
+// and the correctly rounded reciprocal).  Host callable; a host test checks
+// it against IEEE division for every normal fp32 a >= 2^-119 (a / 127 normal).
+__host__ __device__ __forceinline__ float div127_rn(float a) {
+  constexpr float kInv127 = 1.0f / 127.0f;  // RN32(1/127), folded at compile time
+#ifdef __CUDA_ARCH__
+  const float q0 = __fmul_rn(a, kInv127);
+  return __fmaf_rn(__fmaf_rn(-q0, 127.0f, a), kInv127, q0);
+#else
+  const float q0 = a * kInv127;
+  return fmaf(fmaf(-q0, 127.0f, a), kInv127, q0);
+#endif
+}
+
 // Rescale epilogue: s_m = RN32(RN32(eta_m * gamma) / 127) (computed once per
-// token), y = RN32(RN32(float(y_int)) * s_m).  __fmul_rn / __fdiv_rn keep
-// each step a single IEEE rounding (no contraction into an FMA).
+// token), y = RN32(RN32(float(y_int)) * s_m).  Each step is a single IEEE
+// rounding (no contraction into an FMA).
 __device__ __forceinline__ float token_scale(float eta, float gamma) {
-  return __fdiv_rn(__fmul_rn(eta, gamma), 127.0f);
+  return div127_rn(__fmul_rn(eta, gamma));
 }
 
 __device__ __forceinline__ float rescale(int32_t y_int, float s) {

@@ -322,7 +322,8 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode(const DecodeArgs a) {
 #pragma unroll
       for (int i = 0; i < kDecComputeWarps; ++i) e = max(e, T.s_max[i][m]);
       const float eta = fmaxf(__uint_as_float(e), 1e-5f);
-      const float qs = quant_scale(eta);
+      const float rr = rcp_approx(eta);
+      const float qs = __fmul_rn(127.0f, rr);
       const float heta = __fmul_rn(0.5f, eta);
       const bool eta_bf16 = is_bf16_value(eta);
       int32_t psum = 0;
@@ -335,8 +336,8 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode(const DecodeArgs a) {
           const float f2 = __uint_as_float(u.y << 16), f3 = __uint_as_float(u.y & 0xFFFF0000u);
           uint32_t b0, b1, b2, b3;
           if (eta_bf16) {
-            b0 = code_bits_bf16(f0, eta, heta, qs); b1 = code_bits_bf16(f1, eta, heta, qs);
-            b2 = code_bits_bf16(f2, eta, heta, qs); b3 = code_bits_bf16(f3, eta, heta, qs);
+            b0 = code_bits_bf16_r(f0, eta, heta, qs, rr); b1 = code_bits_bf16_r(f1, eta, heta, qs, rr);
+            b2 = code_bits_bf16_r(f2, eta, heta, qs, rr); b3 = code_bits_bf16_r(f3, eta, heta, qs, rr);
           } else {
             b0 = quantise_exact_bits(f0, eta); b1 = quantise_exact_bits(f1, eta);
             b2 = quantise_exact_bits(f2, eta); b3 = quantise_exact_bits(f3, eta);

@@ -10,6 +10,7 @@
 // (sum x~ * t = sum x~ * c - sum x~).
 #pragma once
 
+#include <cstring>
 #include <type_traits>
 
 #include "common.cuh"
@@ -99,6 +100,81 @@ __device__ __forceinline__ uint32_t code_bits_bf16(float x, float eta, float het
   return bits;
 }
 
+// Round-to-nearest fp32 steps callable from host and device, each one IEEE
+// operation (no contraction): the device uses the _rn intrinsics, the host
+// its own IEEE arithmetic (a host build of this header must not contract,
+// e.g. gcc -ffp-contract=off), so the exhaustive host checks of the rules
+// below run the same arithmetic as the kernels.
+__host__ __device__ __forceinline__ float f32_mul(float a, float b) {
+#ifdef __CUDA_ARCH__
+  return __fmul_rn(a, b);
+#else
+  return a * b;
+#endif
+}
+__host__ __device__ __forceinline__ float f32_sub(float a, float b) {
+#ifdef __CUDA_ARCH__
+  return __fsub_rn(a, b);
+#else
+  return a - b;
+#endif
+}
+__host__ __device__ __forceinline__ float f32_fma(float a, float b, float c) {
+#ifdef __CUDA_ARCH__
+  return __fmaf_rn(a, b, c);
+#else
+  return fmaf(a, b, c);
+#endif
+}
+__host__ __device__ __forceinline__ uint32_t f32_bits(float v) {
+#ifdef __CUDA_ARCH__
+  return __float_as_uint(v);
+#else
+  uint32_t u;
+  memcpy(&u, &v, 4);
+  return u;
+#endif
+}
+
+// The bf16 quantiser rule of the kernels: x~ = RNE(RN32(RN32(x*127)/eta))
+// exactly, with no division, from an approximate reciprocal.  x and eta are
+// bf16 values (eta >= 1e-5), heta = eta/2, r approximates 1/eta within
+// 2^-21 relative (rcp.approx has 1 ulp) and s = RN32(127 r).  With
+// q = 127x/eta (|q| <= 127; 127x and the quotient's RN32 keep q's side of
+// every half-integer, see code_bits_bf16):
+//   * t = RN32(x s + M), M = 1.5 * 2^23: t - M = n0 is an integer with
+//     |n0 - q| < 1 (x s is within 127 (2^-21 + 2^-24) < 7e-5 of q);
+//   * e = 127x - n0 eta, exact (one fma; see code_bits_bf16);
+//   * RN32(e r + t) rounds M + n0 + e/eta + err, |err| <= |e/eta| 2^-21 <
+//     2.5e-7, to an integer, and q = n0 + e/eta.  q is either exactly a half-integer or at least
+//     1/(2 * 255 * 2^9) > 3.8e-6 away from every half-integer (the
+//     denominator argument of code_bits_bf16; exponent gaps of 10 or more
+//     leave |q| < 0.25), so the fp32 adder's rounding to an integer is
+//     RNE(q) for every q that is not a tie;
+//   * a tie is exactly |e| = eta/2; then the even one of n0 and n0 + sign(e)
+//     is taken (t's last significand bit is n0's parity).
+// Returns the bit pattern of RNE(q) + M (its low byte is the int8 code).
+__host__ __device__ __forceinline__ uint32_t code_bits_bf16_r(float x, float eta, float heta, float s,
+                                                              float r) {
+  const float t = f32_fma(x, s, kRneMagic);
+  const float n0 = f32_sub(t, kRneMagic);
+  const float e = f32_fma(-n0, eta, f32_mul(x, 127.0f));
+  uint32_t b = f32_bits(f32_fma(e, r, t));
+  if (fabsf(e) == heta) {
+    const uint32_t tb = f32_bits(t);
+    b = (tb & 1u) ? tb + (e > 0.0f ? 1u : 0xFFFFFFFFu) : tb;
+  }
+  return b;
+}
+
+// 1/eta to within 1 ulp (the hardware reciprocal approximation), for the
+// candidate and correction of code_bits_bf16_r.
+__device__ __forceinline__ float rcp_approx(float v) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(v));
+  return r;
+}
+
 // Whether v is a bf16 value (its low 16 bits are zero).
 __device__ __forceinline__ bool is_bf16_value(float v) {
   return (__float_as_uint(v) & 0xFFFFu) == 0;
@@ -108,9 +184,10 @@ __device__ __forceinline__ bool is_bf16_value(float v) {
 // floor rather than a bf16 value (every |x| of the row below 1e-5), the
 // argument above does not hold and the code takes the IEEE quotient
 // (a uniform branch: eta is shared by the row).
-__device__ __forceinline__ int32_t quantise_bf16(float x, float eta, float s, bool eta_bf16) {
-  const uint32_t bits = eta_bf16 ? code_bits_bf16(x, eta, __fmul_rn(0.5f, eta), s)
-                                 : quantise_exact_bits(x, eta);
+// s = RN32(127 r), r = rcp_approx(eta) (see code_bits_bf16_r).
+__device__ __forceinline__ int32_t quantise_bf16(float x, float eta, float heta, float s, float r,
+                                                 bool eta_bf16) {
+  const uint32_t bits = eta_bf16 ? code_bits_bf16_r(x, eta, heta, s, r) : quantise_exact_bits(x, eta);
   return static_cast<int32_t>(bits - kRneMagicBits);
 }
 
@@ -225,14 +302,17 @@ __global__ void __launch_bounds__(256) k_quant_act(const T* __restrict__ x, int6
     }
     amax = block_max_256(amax, redf);
     const float eta = fmaxf(amax, 1e-5f);
-    const float qs = quant_scale(eta);
+    const float qs = kBf16 ? 0.0f : quant_scale(eta);
+    const float rr = kBf16 ? rcp_approx(eta) : 0.0f;
+    const float rs = __fmul_rn(127.0f, rr);
+    const float heta = __fmul_rn(0.5f, eta);
     const bool eta_bf16 = is_bf16_value(eta);
     int32_t sum = 0;
     auto quant_store = [&](int64_t k, const float (&f)[V]) {
       int32_t q[V];
 #pragma unroll
       for (int i = 0; i < V; ++i) {
-        q[i] = kBf16 ? quantise_bf16(f[i], eta, qs, eta_bf16) : quantise_fast(f[i], eta, qs);
+        q[i] = kBf16 ? quantise_bf16(f[i], eta, heta, rs, rr, eta_bf16) : quantise_fast(f[i], eta, qs);
         sum += q[i];
       }
       QVec<T>::store(qrow + k, q);
@@ -251,7 +331,7 @@ __global__ void __launch_bounds__(256) k_quant_act(const T* __restrict__ x, int6
     } else {
       for (int64_t k = threadIdx.x; k < K; k += 256) {
         const float xv = load_as_f32(row + k);
-        const int32_t q = kBf16 ? quantise_bf16(xv, eta, qs, eta_bf16) : quantise_fast(xv, eta, qs);
+        const int32_t q = kBf16 ? quantise_bf16(xv, eta, heta, rs, rr, eta_bf16) : quantise_fast(xv, eta, qs);
         sum += q;
         qrow[k] = static_cast<int8_t>(q);
       }

@@ -1,0 +1,84 @@
+// Host driver for two division-free rules of the kernels, compiled from the
+// kernels' own __host__ __device__ routines (quant.cuh, common.cuh), used by
+// tests/test_fast_rules.py.
+//   quant   : code_bits_bf16_r against RNE(RN32(RN32(127 x) / eta)) (IEEE
+//             division) for every bf16 x with |x| <= eta, eta = every bf16
+//             significand at several exponents, and reciprocals r that are
+//             off RN32(1/eta) by -8..+8 ulps (the rule needs r within
+//             2^-21 relative; the hardware approximation is within 1 ulp).
+//   div127  : div127_rn(a) against the IEEE quotient a / 127 for every
+//             normal fp32 a >= 2^-119.
+// Prints counts; the test requires zero mismatches.
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+
+#include "quant.cuh"
+
+static float from_bits(uint32_t u) {
+  float f;
+  memcpy(&f, &u, 4);
+  return f;
+}
+static uint32_t to_bits(float f) {
+  uint32_t u;
+  memcpy(&u, &f, 4);
+  return u;
+}
+
+static int run_quant() {
+  long long checked = 0, bad = 0, ties = 0;
+  const int exps[] = {-12, -3, 0, 5, 20};
+  for (int E : exps) {
+    for (int m = 128; m < 256; ++m) {
+      const float eta = std::ldexp(static_cast<float>(m) / 128.0f, E);  // a bf16 value
+      const float heta = eta * 0.5f;
+      const float r0 = 1.0f / eta;
+      for (int k = -8; k <= 8; ++k) {
+        const float r = from_bits(to_bits(r0) + k);
+        const float s = bl::f32_mul(127.0f, r);
+        for (uint32_t b = 0; b < 0x7F80u; ++b) {
+          const float v = from_bits(b << 16);
+          if (!(v <= eta)) continue;
+          for (int sg = 0; sg < 2; ++sg) {
+            const float x = sg ? -v : v;
+            volatile float a = x * 127.0f;
+            volatile float q = a / eta;
+            float rq = std::nearbyint(q);
+            rq = std::fmin(127.0f, std::fmax(-127.0f, rq));
+            if (k == 0 && std::fabs(q - std::trunc(q)) == 0.5f) ++ties;
+            const int got = static_cast<int>(bl::code_bits_bf16_r(x, eta, heta, s, r) - bl::kRneMagicBits);
+            bad += (got != static_cast<int>(rq));
+            ++checked;
+          }
+        }
+      }
+    }
+  }
+  printf("quant checked=%lld mismatches=%lld ties=%lld\n", checked, bad, ties);
+  return 0;
+}
+
+static int run_div127() {
+  const uint32_t lo = to_bits(std::ldexp(1.0f, -119)), hi = 0x7F7FFFFFu;
+  long long bad = 0, checked = 0;
+#pragma omp parallel for reduction(+ : bad, checked) schedule(static)
+  for (long long u = lo; u <= static_cast<long long>(hi); ++u) {
+    const float a = from_bits(static_cast<uint32_t>(u));
+    volatile float ref = a / 127.0f;
+    bad += (to_bits(bl::div127_rn(a)) != to_bits(ref));
+    ++checked;
+  }
+  // the constant is the correctly rounded reciprocal
+  const float c = 1.0f / 127.0f;
+  const double e0 = std::fabs(static_cast<double>(c) - 1.0 / 127.0);
+  const double e1 = std::fabs(static_cast<double>(from_bits(to_bits(c) + 1)) - 1.0 / 127.0);
+  const double e2 = std::fabs(static_cast<double>(from_bits(to_bits(c) - 1)) - 1.0 / 127.0);
+  printf("div127 checked=%lld mismatches=%lld inv127_nearest=%d\n", checked, bad, (e0 < e1 && e0 < e2) ? 1 : 0);
+  return 0;
+}
+
+int main(int argc, char** argv) {
+  if (argc > 1 && strcmp(argv[1], "div127") == 0) return run_div127();
+  return run_quant();
+}

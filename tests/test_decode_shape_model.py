@@ -81,3 +81,31 @@ def test_bad_arguments(L):
     assert shape(L, 5, 3200, 8640)[0] == _lib.BL_ERR_UNSUPPORTED
     buf = (ctypes.c_int32 * 10)()
     assert L.bitlinear_decode_shape_for(1, 3200, 8640, 1, 148, None) == _lib.BL_ERR_INVALID_ARG
+
+
+def test_register_kernel_shape_picks():
+    """The one-token register-resident kernel: decode_3b's matrices take it
+    (K=3200 -> N=8640: 4 rows per warp, 7 words per lane, 59 rows per CTA;
+    K=8640 -> N=3200: 2 rows per warp, 17 words per lane, 22 rows per CTA),
+    and shapes beyond its register budget or 64 rows per CTA do not."""
+    L = _lib.lib()
+
+    def reg(K, N, sms=148):
+        buf = (ctypes.c_int32 * 4)()
+        st = L.bitlinear_decode_reg_shape(K, N, sms, buf)
+        return None if st == _lib.BL_ERR_UNSUPPORTED else (st, list(buf))
+
+    assert reg(3200, 8640) == (_lib.BL_OK, [4, 7, 59, 147])
+    assert reg(8640, 3200) == (_lib.BL_OK, [2, 17, 22, 146])
+    assert reg(8192, 1024) == (_lib.BL_OK, [1, 16, 7, 147])
+    assert reg(8192, 28672) is None        # 194 rows per CTA
+    assert reg(28672, 8192) is None        # 56 rows per CTA: 4 rows per warp, more than 8 words per lane
+    assert reg(3232, 100) is None          # K not a multiple of 64
+    for K in range(64, 16384 + 1, 64):
+        for N in (1, 148, 2368, 2369, 4736, 9472, 9473):
+            r = reg(K, N)
+            if r is None:
+                continue
+            rb, nj, rpc, grid = r[1]
+            assert rb in (1, 2, 4) and rpc <= 16 * rb and rb * nj <= 34
+            assert 512 * nj >= K and rpc * grid >= N and (grid - 1) * rpc < N

@@ -1,0 +1,58 @@
+"""Exhaustive host checks of two division-free rules the kernels use.
+
+* The bf16 quantiser (quant.cuh, code_bits_bf16_r): x~ = RNE(RN32(RN32(x*127)
+  /eta)) of [Production] "2. Absmax Dynamic Activation Quantization", formed
+  from an approximate reciprocal and an exact fma residual.  Checked for
+  every bf16 x with |x| <= eta, for every bf16 significand of eta at five
+  exponents, with the reciprocal perturbed by up to 8 ulps either way.
+* The rescale's division by 127 (common.cuh, div127_rn): s = RN32(RN32(eta *
+  gamma) / 127) of [Production] pipeline step 5, by a correctly rounded
+  reciprocal and one fma correction.  Checked against the IEEE quotient for
+  every normal fp32 a >= 2^-119.
+
+Both routines are __host__ __device__; this test compiles them for the host
+with nvcc (no GPU needed; contraction off, as in the kernels).
+"""
+import os
+import re
+import shutil
+import subprocess
+import tempfile
+
+import pytest
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+CSRC = os.path.join(os.path.dirname(HERE), "ternary_weight_linear_04_b200", "csrc")
+
+
+@pytest.fixture(scope="module")
+def driver():
+    nvcc = shutil.which("nvcc") or "/usr/local/cuda/bin/nvcc"
+    if not os.path.exists(nvcc):
+        pytest.skip("nvcc not available")
+    d = tempfile.mkdtemp(prefix="rules_")
+    exe = os.path.join(d, "host_rules")
+    subprocess.run([nvcc, "-O2", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a",
+                    "-Xcompiler", "-ffp-contract=off,-fopenmp", "-I", CSRC, "-o", exe,
+                    os.path.join(HERE, "host_rules.cu"), "-lgomp"],
+                   check=True, capture_output=True)
+    yield exe
+    shutil.rmtree(d, ignore_errors=True)
+
+
+def _counts(out):
+    return {k: int(v) for k, v in re.findall(r"(\w+)=(\d+)", out)}
+
+
+def test_bf16_quantiser_rule_is_exact(driver):
+    c = _counts(subprocess.run([driver, "quant"], check=True, capture_output=True, text=True).stdout)
+    assert c["checked"] > 100_000_000
+    assert c["mismatches"] == 0
+    assert c["ties"] > 100  # exact .5 ties occur, so the tie branch is exercised
+
+
+def test_division_by_127_is_correctly_rounded(driver):
+    c = _counts(subprocess.run([driver, "div127"], check=True, capture_output=True, text=True).stdout)
+    assert c["checked"] > 2_000_000_000
+    assert c["mismatches"] == 0
+    assert c["inv127_nearest"] == 1

@@ -626,3 +626,68 @@ def test_forward3_many_tokens_with_large_shared_memory(M, K):
         y, y_int = bl.forward3(xq, eta, xsum, packed3, gamma, N, out_dtype=DT[out], want_int=True)
         np.testing.assert_array_equal(y_int.cpu().numpy(), ref_yint)
         np.testing.assert_array_equal(y_bits(y.cpu()), oracle_y_bits(ref_y, out))
+
+
+# ----------------------------------------------------------------- one token, weights in registers
+
+_REG_CASES = ([(K, 1000) for K in (1024, 2048, 3200, 4096, 6144, 8192, 8640, 12288)]
+              + [(K, 3200) for K in (1024, 2048, 3200, 4096, 6144, 8192, 8640)]
+              + [(K, 8640) for K in (1024, 2048, 3200, 4096)]
+              + [(64, 5), (3200, 8641), (8640, 2369), (1024, 148), (1024, 149)])
+
+
+@pytest.mark.parametrize("K,N", _REG_CASES)
+def test_register_decode_kernel_every_shape(K, N):
+    """bitlinear_linear for one token on the kernel that holds each CTA's
+    weights in registers: every (rows per warp, words per lane)
+    instantiation, ragged last CTAs (N = 8641, 149), padding words (K = 3200
+    fills 200 of 224 word slots), static and non-static weights, fp32 and
+    bf16 y, y_int and the optional x~ / eta / xsum outputs, all bit-exact
+    against the oracle."""
+    shp = bl.decode_reg_shape(K, N)
+    assert shp is not None, "the register kernel takes (K, N)"
+    W, x = inputs.make_case(12000 + K + N, 1, K, N, act_dtype="bf16")
+    ref_packed, ref_gamma, _ = orc.pack_weights(W)
+    _, _, packed, gamma = gpu_pack(W)
+    ref_xq, ref_eta, ref_xsum = orc.quant_act(x)
+    ref_yint, ref_y = orc.forward(ref_xq, ref_eta, ref_packed, ref_gamma, K, N)
+    xd = torch.from_numpy(x).cuda().to(torch.bfloat16)
+    torch.cuda.synchronize()
+    for static in (True, False):
+        y, (xq, eta, xsum), y_int = bl.linear(xd, packed, gamma, N, out_dtype=torch.bfloat16,
+                                              want_quant=True, want_int=True, weights_static=static)
+        np.testing.assert_array_equal(xq.cpu().numpy(), ref_xq)
+        np.testing.assert_array_equal(eta.cpu().numpy().view(np.uint32), ref_eta.view(np.uint32))
+        np.testing.assert_array_equal(xsum.cpu().numpy(), ref_xsum)
+        np.testing.assert_array_equal(y_int.cpu().numpy(), ref_yint)
+        np.testing.assert_array_equal(y_bits(y.cpu()), orc.f32_to_bf16_bits(ref_y))
+    y32 = bl.linear(xd, packed, gamma, N, out_dtype=torch.float32, weights_static=True)
+    np.testing.assert_array_equal(y32.cpu().numpy().view(np.uint32), ref_y.view(np.uint32))
+
+
+def test_register_decode_kernel_eta_floor_and_forced_ring(forced_shape):
+    """A row with every |x| below 1e-5 (eta is the 1e-5 floor, not a bf16
+    value: the kernel takes IEEE quotients), and the same call with a decode
+    shape forced, which runs the shared-memory kernel instead: identical
+    outputs."""
+    K, N = 3200, 1000
+    rng = np.random.default_rng(12)
+    bits = rng.integers(0x3000, 0x3727, size=(1, K)).astype(np.uint32)
+    x = ((bits << 16).view(np.float32) * np.where(rng.random((1, K)) < 0.5, -1, 1)).astype(np.float32)
+    W, _ = inputs.make_case(12001, 1, K, N)
+    ref_packed, ref_gamma, _ = orc.pack_weights(W)
+    _, _, packed, gamma = gpu_pack(W)
+    ref_xq, ref_eta, ref_xsum = orc.quant_act(x)
+    _, ref_y = orc.forward(ref_xq, ref_eta, ref_packed, ref_gamma, K, N)
+    xd = torch.from_numpy(x).cuda().to(torch.bfloat16)
+    outs = []
+    for force in (False, True):
+        if force:
+            forced_shape(1, 4)
+        y, (xq, eta, xsum) = bl.linear(xd, packed, gamma, N, out_dtype=torch.float32, want_quant=True,
+                                       weights_static=True)
+        np.testing.assert_array_equal(xq.cpu().numpy(), ref_xq)
+        np.testing.assert_array_equal(xsum.cpu().numpy(), ref_xsum)
+        np.testing.assert_array_equal(y.cpu().numpy().view(np.uint32), ref_y.view(np.uint32))
+        outs.append(y.cpu())
+    assert torch.equal(outs[0], outs[1])
