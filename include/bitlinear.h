@@ -346,6 +346,16 @@ bl_status bitlinear_decode_shape_for(int64_t M, int64_t K, int64_t N, int fused,
 bl_status bitlinear_decode_reg_shape(int64_t K, int64_t N, int sms, int32_t* shape);
 
 /*
+ * Turn the one-token register-resident kernel of bitlinear_linear on (1, the
+ * default) or off (0) for every later launch in this process; off, one-token
+ * calls run the shared-memory decode kernel.  Results are identical either
+ * way; this exists to compare the kernels.  No counterpart on the pages.
+ * Not synchronised with launches in flight on other host threads.
+ * Errors: BL_ERR_INVALID_ARG for values other than 0 and 1.
+ */
+bl_status bitlinear_set_decode_reg(int enable);
+
+/*
  * Force the decode kernel's shape for every later launch in this process:
  * team_warps G in 1..16 and rows_per_block RB in {1, 2, 4, 8, 16} (RB * M'
  * <= 16 with M' = M rounded up to 1, 2 or 4); 0 for either leaves that

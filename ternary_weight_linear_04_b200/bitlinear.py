@@ -187,6 +187,12 @@ def decode_reg_shape(K, N, sms=None):
     return dict(zip(("rows_per_warp", "words_per_lane", "rows_per_cta", "ctas"), list(buf)))
 
 
+def set_decode_reg(enable=True):
+    """Turn the one-token register-resident kernel on (default) or off for
+    later launches in this process (off: the shared-memory decode kernel)."""
+    check(_lib.lib().bitlinear_set_decode_reg(1 if enable else 0), "bitlinear_set_decode_reg")
+
+
 def set_tc_split(k_split=0):
     """Force the K split (CTAs per cluster) of the tensor-core kernel for later
     launches in this process (0 = the library's choice)."""

@@ -220,6 +220,8 @@ inline bool rb_allowed(int MT, int RB) { return RB * MT <= 16; }
 
 // Shape forced by bitlinear_set_decode_shape (0 = chosen by the model).
 std::atomic<int> g_force_G{0}, g_force_RB{0};
+// bitlinear_set_decode_reg: 0 turns the one-token register-resident kernel off.
+std::atomic<int> g_decode_reg{1};
 
 bool decode_geometry(int MT, int64_t M, int64_t K, int64_t N, int sms, int64_t xelem,
                      DecGeom* out) {
@@ -402,7 +404,7 @@ struct RegGeom {
 };
 
 constexpr int kRegNJ1[] = {2, 4, 7, 8, 12, 16, 17, 24};
-constexpr int kRegNJ2[] = {2, 4, 7, 8, 12, 16, 17};
+constexpr int kRegNJ2[] = {2, 4, 7, 8, 12, 17};
 constexpr int kRegNJ4[] = {2, 4, 7, 8};
 
 bool reg_decode_geometry(int64_t K, int64_t N, int sms, RegGeom* g) {
@@ -414,7 +416,7 @@ bool reg_decode_geometry(int64_t K, int64_t N, int sms, RegGeom* g) {
   if (RB == 0) return false;
   const int64_t need = (K / 16 + 31) / 32;
   const int* list = RB == 1 ? kRegNJ1 : (RB == 2 ? kRegNJ2 : kRegNJ4);
-  const int n = RB == 1 ? 8 : (RB == 2 ? 7 : 4);
+  const int n = RB == 1 ? 8 : (RB == 2 ? 6 : 4);
   int NJ = 0;
   for (int i = 0; i < n && !NJ; ++i)
     if (list[i] >= need) NJ = list[i];
@@ -441,7 +443,7 @@ bl_status launch_decode_reg(const bl::RegDecodeArgs& a, const RegGeom& g, cudaSt
   BL_REG_CASE(1, 2) BL_REG_CASE(1, 4) BL_REG_CASE(1, 7) BL_REG_CASE(1, 8) BL_REG_CASE(1, 12)
   BL_REG_CASE(1, 16) BL_REG_CASE(1, 17) BL_REG_CASE(1, 24)
   BL_REG_CASE(2, 2) BL_REG_CASE(2, 4) BL_REG_CASE(2, 7) BL_REG_CASE(2, 8) BL_REG_CASE(2, 12)
-  BL_REG_CASE(2, 16) BL_REG_CASE(2, 17)
+  BL_REG_CASE(2, 17)
   BL_REG_CASE(4, 2) BL_REG_CASE(4, 4) BL_REG_CASE(4, 7) BL_REG_CASE(4, 8)
 #undef BL_REG_CASE
   return BL_ERR_UNSUPPORTED;
@@ -703,6 +705,12 @@ bl_status bitlinear_decode_reg_shape(int64_t K, int64_t N, int sms, int32_t* sha
   shape[1] = g.NJ;
   shape[2] = g.rows_per_cta;
   shape[3] = g.grid;
+  return BL_OK;
+}
+
+bl_status bitlinear_set_decode_reg(int enable) {
+  if (enable != 0 && enable != 1) return BL_ERR_INVALID_ARG;
+  g_decode_reg.store(enable, std::memory_order_relaxed);
   return BL_OK;
 }
 
@@ -1035,7 +1043,8 @@ bl_status bitlinear_linear(const void* x, bl_dtype xdt, int64_t M, int64_t K, co
   // One token: the register-resident kernel when the CTA's share fits (and
   // no decode shape is forced for the shared-memory kernel).
   RegGeom rg;
-  if (M == 1 && g_force_G.load(std::memory_order_relaxed) == 0 &&
+  if (M == 1 && g_decode_reg.load(std::memory_order_relaxed) != 0 &&
+      g_force_G.load(std::memory_order_relaxed) == 0 &&
       g_force_RB.load(std::memory_order_relaxed) == 0 && reg_decode_geometry(K, N, sms, &rg)) {
     bl::RegDecodeArgs r = {};
     r.x = static_cast<const __nv_bfloat16*>(x);

@@ -262,11 +262,20 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode(const DecodeArgs a) {
     __syncwarp();
     named_arrive(3, kDecThreads);  // barriers initialised, gamma in place, inputs readable
     if (lane == 0) {
+      int issued = first;
       for (int c = S; c < nchunks; ++c) {
         const int s = c % S;
         if (!mbar_wait(&T.empty[s], static_cast<uint32_t>(c / S - 1) & 1u, &T.abort_flag)) break;
         issue(c);
+        issued = c + 1;
       }
+      // Before this warp exits, the copies it issued have landed (bounded
+      // waits): after an abort nothing may still be writing into shared
+      // memory when the CTA ends.  In the normal flow they have already
+      // been consumed, or land shortly, and the waits return at once.
+      for (int c = issued > S ? issued - S : 0; c < issued; ++c)
+        mbar_drain(&T.full[c % S], static_cast<uint32_t>(c / S) & 1u);
+      if (a.x_staged) mbar_drain(&T.xfull, 0);
     }
     return;
   }

@@ -26,8 +26,16 @@
 //     matching slot words, sum x~ c - sum x~ = sum x~ t), then a transposed
 //     warp reduction leaves each row total on one lane, which rescales and
 //     stores it.
-// 512 threads and at most 64 registers each, so the next layer's CTA fits on
-// the SM beside this one under programmatic dependent launch.
+// 512 threads and at most 56 registers each (the launch bound names 576
+// threads so that the compiler keeps to 56): the next layer's CTA must fit
+// on the SM beside this one under programmatic dependent launch, and the
+// register file is split over four sub-partitions of 16K registers, each
+// holding a quarter of a CTA's warps.  The shared-memory decode kernel puts
+// five of its 17 warps (56 registers) on one sub-partition, 8960
+// registers; four warps of this kernel at 64 registers (8192) would not fit
+// beside them, at 56 (7168) they do.  Measured on a 70B-class layer's seven
+// projections chained under dependent launch: 104 us with the cap, 142 us at
+// 64 registers (every switch between the two kernels then lost the overlap).
 #pragma once
 
 #include "common.cuh"
@@ -76,7 +84,7 @@ __device__ __forceinline__ uint32_t ld_nc_na_u32(const void* p) {
 // NJ words per lane and row (K <= 512 NJ), RB rows per warp.  Shared
 // memory: 32 NJ slots of 16 bytes.
 template <int RB, int NJ>
-__global__ void __launch_bounds__(kRegThreads, 2) k_decode_reg(const RegDecodeArgs a) {
+__global__ void __launch_bounds__(kRegThreads + 64, 2) k_decode_reg(const RegDecodeArgs a) {
   static_assert(RB == 1 || RB == 2 || RB == 4, "RB rows per warp: 1, 2 or 4");
   constexpr int XC = (NJ + 7) / 8;  // 16-byte chunks of x per thread
   extern __shared__ __align__(16) uint8_t smem[];
