@@ -346,10 +346,29 @@ bl_status bitlinear_decode_shape_for(int64_t M, int64_t K, int64_t N, int fused,
 bl_status bitlinear_decode_reg_shape(int64_t K, int64_t N, int sms, int32_t* shape);
 
 /*
- * Turn the one-token register-resident kernel of bitlinear_linear on (1, the
- * default) or off (0) for every later launch in this process; off, one-token
- * calls run the shared-memory decode kernel.  Results are identical either
- * way; this exists to compare the kernels.  No counterpart on the pages.
+ * Shape of the register-resident kernel for 2 to 4 tokens whose x~ is given
+ * (BL_PATH_GEMV of bitlinear_forward, and the accumulate step of
+ * bitlinear_linear from 3 tokens on), for M tokens, K inputs and N outputs
+ * on a GPU with `sms` SMs (host logic only; usable without a GPU).  The
+ * pages have no counterpart.  The library uses this kernel for 2 <= M <= 4
+ * on the decode path when this query succeeds and no decode shape is forced
+ * (bitlinear_set_decode_shape); otherwise the shared-memory decode kernel.
+ * shape (host, 5 int32) receives: token slots MT (2 or 4), rows per warp RB
+ * (16 warps per CTA), 32-bit weight words per lane and row NJ (K <= 512 NJ),
+ * rows per CTA, CTAs.  Errors: BL_ERR_INVALID_ARG for shape == NULL, K < 1,
+ * N < 1 or sms < 1; BL_ERR_UNSUPPORTED when the kernel does not take
+ * (M, K, N): M outside 2..4, K not a multiple of 64, more than 64 rows per
+ * CTA, RB * MT above 16, or more weight words than its register budget.
+ */
+bl_status bitlinear_decode_regm_shape(int64_t M, int64_t K, int64_t N, int sms, int32_t* shape);
+
+/*
+ * Turn the register-resident kernels on (1, the default) or off (0) for
+ * every later launch in this process: the one-token kernel of
+ * bitlinear_linear (quantiser fused) and the 2..4-token kernel of the
+ * decode path (x~ given).  Off, those calls run the shared-memory decode
+ * kernel.  Results are identical either way; this exists to compare the
+ * kernels.  No counterpart on the pages.
  * Not synchronised with launches in flight on other host threads.
  * Errors: BL_ERR_INVALID_ARG for values other than 0 and 1.
  */

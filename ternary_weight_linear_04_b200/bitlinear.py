@@ -187,9 +187,24 @@ def decode_reg_shape(K, N, sms=None):
     return dict(zip(("rows_per_warp", "words_per_lane", "rows_per_cta", "ctas"), list(buf)))
 
 
+def decode_regm_shape(M, K, N, sms=None):
+    """Shape of the register-resident kernel for 2..4 tokens with x~ given,
+    as a dict, or None when that kernel does not take (M, K, N).  sms
+    defaults to the current device's SM count."""
+    if sms is None:
+        sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    buf = (ctypes.c_int32 * 5)()
+    st = _lib.lib().bitlinear_decode_regm_shape(M, K, N, sms, buf)
+    if st == _lib.BL_ERR_UNSUPPORTED:
+        return None
+    check(st, "bitlinear_decode_regm_shape")
+    return dict(zip(("token_slots", "rows_per_warp", "words_per_lane", "rows_per_cta", "ctas"), list(buf)))
+
+
 def set_decode_reg(enable=True):
-    """Turn the one-token register-resident kernel on (default) or off for
-    later launches in this process (off: the shared-memory decode kernel)."""
+    """Turn the register-resident kernels (one token fused; 2..4 tokens with
+    x~ given) on (default) or off for later launches in this process (off:
+    the shared-memory decode kernel)."""
     check(_lib.lib().bitlinear_set_decode_reg(1 if enable else 0), "bitlinear_set_decode_reg")
 
 

@@ -141,7 +141,14 @@ bool ensure_smem(Kern kern, size_t bytes, int* done_flags) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
   if (done_flags[dev] >= static_cast<int>(bytes) && done_flags[dev] > 0) return true;
-  if (bytes > 48 * 1024 &&
+  // The default limit (48 KB) covers static and dynamic shared memory
+  // together: raise the dynamic limit whenever the sum would pass it.
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return false;
+  }
+  if (bytes + fa.sharedSizeBytes > 48 * 1024 &&
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(bytes)) != cudaSuccess) {
     (void)cudaGetLastError();  // do not leave the error for the next launch check
@@ -220,7 +227,8 @@ inline bool rb_allowed(int MT, int RB) { return RB * MT <= 16; }
 
 // Shape forced by bitlinear_set_decode_shape (0 = chosen by the model).
 std::atomic<int> g_force_G{0}, g_force_RB{0};
-// bitlinear_set_decode_reg: 0 turns the one-token register-resident kernel off.
+// bitlinear_set_decode_reg: 0 turns the register-resident kernels off (one
+// token fused with the quantiser; 2..4 tokens with x~ given).
 std::atomic<int> g_decode_reg{1};
 
 bool decode_geometry(int MT, int64_t M, int64_t K, int64_t N, int sms, int64_t xelem,
@@ -449,6 +457,66 @@ bl_status launch_decode_reg(const bl::RegDecodeArgs& a, const RegGeom& g, cudaSt
   return BL_ERR_UNSUPPORTED;
 }
 
+// Register-resident kernel for 2..4 tokens with x~ given (decode_reg.cuh):
+// the rows of the one-token geometry (one CTA per SM, RB rows per warp), MT
+// = 2 or 4 token slots, and the smallest instantiated word count NJ that
+// covers K.  The instantiated (MT, RB, NJ) keep weights, RB * MT
+// accumulators and two activation slots within 64 registers with no spills
+// (ptxas), which leaves room for two CTAs per SM.
+struct RegMGeom {
+  int MT = 0, RB = 0, NJ = 0, rows_per_cta = 0, grid = 0;
+};
+
+constexpr int kRegMNJ1[] = {2, 4, 7, 8, 12, 17, 24};
+constexpr int kRegMNJ2[] = {2, 4, 7, 8, 12, 17};
+constexpr int kRegMNJ4[] = {2, 4, 7, 8};
+
+bool regm_geometry(int64_t M, int64_t K, int64_t N, int sms, RegMGeom* g) {
+  if (M < 2 || M > bl::kRegMultiMaxMT) return false;
+  RegGeom g1;
+  if (!reg_decode_geometry(K, N, sms, &g1)) return false;
+  const int MT = M <= 2 ? 2 : 4;
+  if (g1.RB * MT > 16) return false;
+  const int64_t need = (K / 16 + 31) / 32;
+  const int* list = g1.RB == 1 ? kRegMNJ1 : (g1.RB == 2 ? kRegMNJ2 : kRegMNJ4);
+  const int n = g1.RB == 1 ? 7 : (g1.RB == 2 ? 6 : 4);
+  int NJ = 0;
+  for (int i = 0; i < n && !NJ; ++i)
+    if (list[i] >= need) NJ = list[i];
+  if (!NJ) return false;
+  g->MT = MT;
+  g->RB = g1.RB;
+  g->NJ = NJ;
+  g->rows_per_cta = g1.rows_per_cta;
+  g->grid = g1.grid;
+  return true;
+}
+
+template <int MT, int RB, int NJ>
+bl_status launch_decode_regm_nj(const bl::RegMultiArgs& a, const RegMGeom& g, cudaStream_t st) {
+  static int done[kMaxDevices] = {0};
+  auto kern = bl::k_decode_regm<MT, RB, NJ>;
+  const size_t smem = static_cast<size_t>(MT) * 32 * NJ * 16;
+  if (!ensure_smem(kern, smem, done)) return BL_ERR_CUDA;
+  return launch_pdl(kern, dim3(static_cast<unsigned>(g.grid)), dim3(bl::kRegThreads), smem, st, a);
+}
+
+bl_status launch_decode_regm(const bl::RegMultiArgs& a, const RegMGeom& g, cudaStream_t st) {
+#define BL_REGM_CASE(T, R, J) \
+  if (g.MT == T && g.RB == R && g.NJ == J) return launch_decode_regm_nj<T, R, J>(a, g, st);
+#define BL_REGM_MT(T)                                                                              \
+  BL_REGM_CASE(T, 1, 2) BL_REGM_CASE(T, 1, 4) BL_REGM_CASE(T, 1, 7) BL_REGM_CASE(T, 1, 8)          \
+  BL_REGM_CASE(T, 1, 12) BL_REGM_CASE(T, 1, 17) BL_REGM_CASE(T, 1, 24)                             \
+  BL_REGM_CASE(T, 2, 2) BL_REGM_CASE(T, 2, 4) BL_REGM_CASE(T, 2, 7) BL_REGM_CASE(T, 2, 8)          \
+  BL_REGM_CASE(T, 2, 12) BL_REGM_CASE(T, 2, 17)                                                    \
+  BL_REGM_CASE(T, 4, 2) BL_REGM_CASE(T, 4, 4) BL_REGM_CASE(T, 4, 7) BL_REGM_CASE(T, 4, 8)
+  BL_REGM_MT(2)
+  BL_REGM_MT(4)
+#undef BL_REGM_MT
+#undef BL_REGM_CASE
+  return BL_ERR_UNSUPPORTED;
+}
+
 template <typename OutT>
 bl_status launch_generic(const int8_t* xq, const float* eta, int64_t M, int64_t K,
                          const uint8_t* packed, const float* gamma, int64_t N, void* y,
@@ -579,6 +647,22 @@ bl_status forward_impl(const int8_t* xq, const float* eta, const int32_t* xsum, 
     if (!fast_layout_ok(K, xq, packed, y, y_int) || !decode_ok(M, K) ||
         N > INT32_MAX / 2)
       return BL_ERR_UNSUPPORTED;
+    // 2..4 tokens: the register-resident kernel when the CTA's share fits
+    // (and no shape is forced for the shared-memory kernel).
+    RegMGeom mg;
+    if (M >= 2 && g_decode_reg.load(std::memory_order_relaxed) != 0 &&
+        g_force_G.load(std::memory_order_relaxed) == 0 &&
+        g_force_RB.load(std::memory_order_relaxed) == 0 && regm_geometry(M, K, N, sms, &mg)) {
+      bl::RegMultiArgs r = {};
+      r.xq = xq; r.eta = eta; r.xsum = xsum;
+      r.M = static_cast<int>(M); r.K = static_cast<int>(K); r.N = static_cast<int>(N);
+      r.packed = packed; r.gamma = gamma; r.y = y;
+      r.y_bf16 = ydt == BL_BF16 ? 1 : 0;
+      r.y_int = y_int;
+      r.rows_per_cta = mg.rows_per_cta;
+      r.weights_static = (flags & BL_FLAG_WEIGHTS_STATIC) ? 1 : 0;
+      return launch_decode_regm(r, mg, s);
+    }
     bl::DecodeArgs a = {};
     a.x = xq; a.eta = eta; a.xsum = xsum; a.M = (int)M; a.K = (int)K; a.N = (int)N;
     a.packed = packed; a.gamma = gamma; a.y = y; a.y_int = y_int;
@@ -694,6 +778,18 @@ bl_status bitlinear_decode_shape(int64_t M, int64_t K, int64_t N, int fused, int
   shape[7] = g.stages;
   shape[8] = g.x_staged;
   shape[9] = static_cast<int32_t>(g.smem);
+  return BL_OK;
+}
+
+bl_status bitlinear_decode_regm_shape(int64_t M, int64_t K, int64_t N, int sms, int32_t* shape) {
+  if (!shape || K < 1 || N < 1 || sms < 1) return BL_ERR_INVALID_ARG;
+  RegMGeom g;
+  if (!regm_geometry(M, K, N, sms, &g)) return BL_ERR_UNSUPPORTED;
+  shape[0] = g.MT;
+  shape[1] = g.RB;
+  shape[2] = g.NJ;
+  shape[3] = g.rows_per_cta;
+  shape[4] = g.grid;
   return BL_OK;
 }
 

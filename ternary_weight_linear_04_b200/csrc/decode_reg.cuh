@@ -238,4 +238,156 @@ __global__ void __launch_bounds__(kRegThreads + 64, 2) k_decode_reg(const RegDec
   }
 }
 
+// ---------------------------------------------------------------------------
+// The same register-resident layout for 2 to 4 tokens whose x~, eta and
+// xsum are given (the quantiser ran before, or the caller passes x~):
+// [Production] "The MatMul-Free Breakthrough" and pipeline step 5 for a few
+// decode tokens at once.
+//   * weights as above: RB rows per warp, NJ words per lane and row, loaded
+//     before griddepcontrol.wait when static;
+//   * after the wait every thread stages its share of the MT x~ rows (all
+//     16-byte loads issued together) into transposed slots, one set per
+//     token; rows past M and words past K/16 are zeros;
+//   * per word, the tokens go in pairs: two slot loads, then for each row the
+//     four planes (w >> 2i) & 0x03030303 (code 4b + i in byte b, matching slot
+//     word i) and 8 dp4a.  The planes are recomputed per pair rather than
+//     kept, which holds the registers to weights + RB * MT accumulators + two
+//     slots (up to 90 at the instantiated shapes, no spills).  One CTA per
+//     SM: in a decode layer the next launch is the quantiser's few CTAs,
+//     which fit beside it, and this kernel's weights stream while they run;
+//   * a transposed warp sum over the RB * MT values leaves each (row, token)
+//     total on one lane, which subtracts xsum, rescales and stores it.
+struct RegMultiArgs {
+  const int8_t* xq;        // M x K
+  const float* eta;        // M
+  const int32_t* xsum;     // M
+  int M, K, N;
+  const uint8_t* packed;
+  const float* gamma;
+  void* y;                 // M x N, fp32 or bf16 (y_bf16)
+  int y_bf16;
+  int32_t* y_int;          // optional
+  int rows_per_cta;        // <= 16 * RB
+  int weights_static;
+};
+
+constexpr int kRegMultiMaxMT = 4;
+
+// MT tokens (2 or 4; M <= MT), RB rows per warp (RB * MT <= 16), NJ words per
+// lane and row.  Shared memory: MT * 32 NJ slots of 16 bytes.
+template <int MT, int RB, int NJ>
+__global__ void __launch_bounds__(kRegThreads, 1) k_decode_regm(const RegMultiArgs a) {
+  static_assert(MT == 2 || MT == 4, "2 or 4 tokens");
+  static_assert(RB == 1 || RB == 2 || RB == 4, "RB rows per warp: 1, 2 or 4");
+  constexpr int NWP = 32 * NJ;                           // slot words per token
+  constexpr int XI = (MT * NWP + kRegThreads - 1) / kRegThreads;  // slots per thread
+  extern __shared__ __align__(16) uint8_t smem[];
+  __shared__ float s_scale[MT];
+  __shared__ int32_t s_xsum[MT];
+  uint4* xslot = reinterpret_cast<uint4*>(smem);
+  const int K = a.K, NW = K >> 4, P = K >> 2, M = a.M;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int r_begin = blockIdx.x * a.rows_per_cta;
+  const int nrows = max(0, min(a.N - r_begin, a.rows_per_cta));
+  const int row0 = warp * RB;
+
+  uint32_t wreg[RB][NJ];
+  auto load_weights = [&]() {
+#pragma unroll
+    for (int r = 0; r < RB; ++r) {
+      const int row = min(row0 + r, max(nrows - 1, 0));
+      const uint8_t* rp = a.packed + static_cast<int64_t>(r_begin + row) * P;
+#pragma unroll
+      for (int j = 0; j < NJ; ++j) {
+        const int wi = lane + 32 * j;
+        wreg[r][j] = (nrows > 0 && wi < NW) ? ld_nc_na_u32(rp + 4 * wi) : 0x55555555u;
+      }
+    }
+  };
+  float gamma = 0.0f;
+  if (a.weights_static) {
+    load_weights();
+    gamma = __ldg(a.gamma);
+  }
+  pdl_wait();  // the previous kernel is complete and its writes are visible
+  if (tid == 0) pdl_trigger();
+  if (!a.weights_static) {
+    load_weights();
+    gamma = __ldg(a.gamma);
+  }
+
+  // x~ slots: slot q = m * NWP + w holds the 16 activations of word w of
+  // token m, transposed (byte b of slot word i = activation 16 w + 4 b + i).
+  {
+    uint4 v[XI];
+#pragma unroll
+    for (int i = 0; i < XI; ++i) {
+      const int q = tid + kRegThreads * i;
+      const int m = q / NWP, w = q - m * NWP;
+      v[i] = (q < MT * NWP && m < M && w < NW)
+                 ? __ldg(reinterpret_cast<const uint4*>(a.xq + static_cast<int64_t>(m) * K) + w)
+                 : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int i = 0; i < XI; ++i) {
+      const int q = tid + kRegThreads * i;
+      if (q < MT * NWP) {
+        uint4 t;
+        transpose4x4_bytes(v[i].x, v[i].y, v[i].z, v[i].w, t.x, t.y, t.z, t.w);
+        xslot[q] = t;
+      }
+    }
+  }
+  if (tid < MT) {
+    s_scale[tid] = tid < M ? token_scale(a.eta[tid], gamma) : 0.0f;
+    s_xsum[tid] = tid < M ? a.xsum[tid] : 0;
+  }
+  __syncthreads();
+  if (row0 >= nrows) return;  // whole warps
+
+  constexpr int V = RB * MT;
+  int32_t acc[V];
+#pragma unroll
+  for (int i = 0; i < V; ++i) acc[i] = 0;
+#pragma unroll
+  for (int j = 0; j < NJ; ++j) {
+#pragma unroll
+    for (int mp = 0; mp < MT; mp += 2) {
+      const uint4 xa = xslot[mp * NWP + lane + 32 * j];
+      const uint4 xb = xslot[(mp + 1) * NWP + lane + 32 * j];
+#pragma unroll
+      for (int r = 0; r < RB; ++r) {
+        const uint32_t w = wreg[r][j];
+        const int p0 = static_cast<int>(w & 0x03030303u);
+        const int p1 = static_cast<int>((w >> 2) & 0x03030303u);
+        const int p2 = static_cast<int>((w >> 4) & 0x03030303u);
+        const int p3 = static_cast<int>((w >> 6) & 0x03030303u);
+        int32_t ta = acc[r * MT + mp], tb = acc[r * MT + mp + 1];
+        ta = __dp4a(p0, static_cast<int>(xa.x), ta);
+        tb = __dp4a(p0, static_cast<int>(xb.x), tb);
+        ta = __dp4a(p1, static_cast<int>(xa.y), ta);
+        tb = __dp4a(p1, static_cast<int>(xb.y), tb);
+        ta = __dp4a(p2, static_cast<int>(xa.z), ta);
+        tb = __dp4a(p2, static_cast<int>(xb.z), tb);
+        ta = __dp4a(p3, static_cast<int>(xa.w), ta);
+        tb = __dp4a(p3, static_cast<int>(xb.w), tb);
+        acc[r * MT + mp] = ta;
+        acc[r * MT + mp + 1] = tb;
+      }
+    }
+  }
+  const int32_t tot = warp_transpose_sum<V>(acc, lane);
+  constexpr int kGroup = 32 / V;
+  const int vi = lane >> ilog2(kGroup);  // value held: row vi / MT, token vi % MT
+  const int r = vi / MT, m = vi - r * MT;
+  if ((lane & (kGroup - 1)) == 0 && row0 + r < nrows && m < M) {
+    const int32_t yi = tot - s_xsum[m];
+    const int64_t o = static_cast<int64_t>(m) * a.N + r_begin + row0 + r;
+    const float yv = rescale(yi, s_scale[m]);
+    if (a.y_bf16) store_out<__nv_bfloat16>(a.y, o, yv);
+    else store_out<float>(a.y, o, yv);
+    if (a.y_int) a.y_int[o] = yi;
+  }
+}
+
 }  // namespace bl

@@ -691,3 +691,65 @@ def test_register_decode_kernel_eta_floor_and_forced_ring(forced_shape):
         np.testing.assert_array_equal(y.cpu().numpy().view(np.uint32), ref_y.view(np.uint32))
         outs.append(y.cpu())
     assert torch.equal(outs[0], outs[1])
+
+
+# ----------------------------------------------------------------- 2..4 tokens, weights in registers
+
+_REGM_CASES = ([(K, 1000) for K in (1024, 2048, 3200, 4096, 6144, 8640, 12288)]
+               + [(K, 3200) for K in (1024, 2048, 3200, 4096, 6144, 8640)]
+               + [(K, 8640) for K in (1024, 2048, 3200, 4096)]
+               + [(64, 5), (3200, 8641), (8640, 2369), (1024, 149)])
+
+
+@pytest.fixture
+def register_kernels():
+    yield bl.set_decode_reg
+    bl.set_decode_reg(True)
+
+
+@pytest.mark.parametrize("M", [2, 3, 4])
+@pytest.mark.parametrize("K,N", _REGM_CASES)
+def test_multi_token_register_kernel_every_shape(register_kernels, M, K, N):
+    """bitlinear_forward (x~ given) for 2..4 tokens on the kernel that holds
+    each CTA's weights in registers: every (token slots, rows per warp, words
+    per lane) instantiation, ragged last CTAs, padding words and tokens (M =
+    3 in 4 slots), static and non-static weights, fp32 and bf16 y; y_int and
+    y bit-exact against the oracle, and identical to the shared-memory
+    decode kernel (register kernels off)."""
+    shp = bl.decode_regm_shape(M, K, N)
+    assert shp is not None, "the register kernel takes (M, K, N)"
+    W, x = inputs.make_case(13000 + 7 * M + K + N, M, K, N, act_dtype="bf16")
+    ref_packed, ref_gamma, _ = orc.pack_weights(W)
+    _, _, packed, gamma = gpu_pack(W)
+    ref_xq, ref_eta, ref_xsum = orc.quant_act(x)
+    ref_yint, ref_y = orc.forward(ref_xq, ref_eta, ref_packed, ref_gamma, K, N)
+    xq, eta, xsum = (torch.from_numpy(a).cuda() for a in (ref_xq, ref_eta, ref_xsum.astype(np.int32)))
+    for static in (True, False):
+        for out in ("bf16", "f32"):
+            y, y_int = bl.forward(xq, eta, xsum, packed, gamma, N, out_dtype=DT[out], want_int=True,
+                                  path="gemv", weights_static=static)
+            np.testing.assert_array_equal(y_int.cpu().numpy(), ref_yint)
+            np.testing.assert_array_equal(y_bits(y.cpu()), oracle_y_bits(ref_y, out))
+    register_kernels(False)
+    y_ring = bl.forward(xq, eta, xsum, packed, gamma, N, out_dtype=torch.bfloat16, path="gemv")
+    np.testing.assert_array_equal(y_bits(y_ring.cpu()), orc.f32_to_bf16_bits(ref_y))
+
+
+@pytest.mark.parametrize("M", [3, 4])
+@pytest.mark.parametrize("K,N", [(3200, 8640), (8640, 3200)])
+def test_multi_token_linear_uses_quantiser_then_register_kernel(M, K, N):
+    """bitlinear_linear for 3..4 tokens (quantiser, then the register kernel)
+    on decode_3b's matrices: x~, eta, xsum, y_int and y bit-exact."""
+    W, x = inputs.make_case(13500 + M + K, M, K, N, act_dtype="bf16")
+    ref_packed, ref_gamma, _ = orc.pack_weights(W)
+    _, _, packed, gamma = gpu_pack(W)
+    ref_xq, ref_eta, ref_xsum = orc.quant_act(x)
+    ref_yint, ref_y = orc.forward(ref_xq, ref_eta, ref_packed, ref_gamma, K, N)
+    xd = torch.from_numpy(x).cuda().to(torch.bfloat16)
+    y, (xq, eta, xsum), y_int = bl.linear(xd, packed, gamma, N, out_dtype=torch.bfloat16, want_quant=True,
+                                          want_int=True, weights_static=True)
+    np.testing.assert_array_equal(xq.cpu().numpy(), ref_xq)
+    np.testing.assert_array_equal(eta.cpu().numpy().view(np.uint32), ref_eta.view(np.uint32))
+    np.testing.assert_array_equal(xsum.cpu().numpy(), ref_xsum)
+    np.testing.assert_array_equal(y_int.cpu().numpy(), ref_yint)
+    np.testing.assert_array_equal(y_bits(y.cpu()), orc.f32_to_bf16_bits(ref_y))
