@@ -260,8 +260,10 @@ bl_status bitlinear_forward(const int8_t* xq, const float* eta, const int32_t* x
  * bitlinear_forward with the accumulate kernel and flags chosen by the
  * caller.  BL_PATH_GEMV and BL_PATH_TCGEN05 return BL_ERR_UNSUPPORTED when
  * the inputs do not meet their layout needs (K % 64 == 0, 16-byte
- * alignment; for BL_PATH_GEMV also M <= 4 and K * M' <= 131072, M' = M
- * rounded up to 1, 2 or 4); the results of every path are identical.
+ * alignment; for BL_PATH_GEMV also either M <= 4 and K * M' <= 131072,
+ * M' = M rounded up to 1, 2 or 4, or 2 <= M <= 8 with a shape the
+ * register-resident kernel takes, see bitlinear_decode_regm_shape); the
+ * results of every path are identical.
  * flags: 0 or BL_FLAG_WEIGHTS_STATIC.
  */
 bl_status bitlinear_forward_path(const int8_t* xq, const float* eta, const int32_t* xsum,
@@ -346,26 +348,27 @@ bl_status bitlinear_decode_shape_for(int64_t M, int64_t K, int64_t N, int fused,
 bl_status bitlinear_decode_reg_shape(int64_t K, int64_t N, int sms, int32_t* shape);
 
 /*
- * Shape of the register-resident kernel for 2 to 4 tokens whose x~ is given
+ * Shape of the register-resident kernel for 2 to 8 tokens whose x~ is given
  * (BL_PATH_GEMV of bitlinear_forward, and the accumulate step of
  * bitlinear_linear from 3 tokens on), for M tokens, K inputs and N outputs
  * on a GPU with `sms` SMs (host logic only; usable without a GPU).  The
- * pages have no counterpart.  The library uses this kernel for 2 <= M <= 4
+ * pages have no counterpart.  The library uses this kernel for 2 <= M <= 8
  * on the decode path when this query succeeds and no decode shape is forced
- * (bitlinear_set_decode_shape); otherwise the shared-memory decode kernel.
- * shape (host, 5 int32) receives: token slots MT (2 or 4), rows per warp RB
+ * (bitlinear_set_decode_shape); otherwise the shared-memory decode kernel
+ * (M <= 4) or the tensor-core kernel (BL_PATH_AUTO, M > 4).
+ * shape (host, 5 int32) receives: token slots MT (2, 4 or 8), rows per warp RB
  * (16 warps per CTA), 32-bit weight words per lane and row NJ (K <= 512 NJ),
  * rows per CTA, CTAs.  Errors: BL_ERR_INVALID_ARG for shape == NULL, K < 1,
  * N < 1 or sms < 1; BL_ERR_UNSUPPORTED when the kernel does not take
- * (M, K, N): M outside 2..4, K not a multiple of 64, more than 64 rows per
- * CTA, RB * MT above 16, or more weight words than its register budget.
+ * (M, K, N): M outside 2..8, K not a multiple of 64, more than 64 rows per
+ * CTA, RB * MT above 32, or more weight words than its register budget.
  */
 bl_status bitlinear_decode_regm_shape(int64_t M, int64_t K, int64_t N, int sms, int32_t* shape);
 
 /*
  * Turn the register-resident kernels on (1, the default) or off (0) for
  * every later launch in this process: the one-token kernel of
- * bitlinear_linear (quantiser fused) and the 2..4-token kernel of the
+ * bitlinear_linear (quantiser fused) and the 2..8-token kernel of the
  * decode path (x~ given).  Off, those calls run the shared-memory decode
  * kernel.  Results are identical either way; this exists to compare the
  * kernels.  No counterpart on the pages.
@@ -473,7 +476,9 @@ bl_status bitlinear_forward3(const int8_t* xq, const float* eta, const int32_t* 
                              int64_t K, const uint8_t* packed3, const float* gamma, int64_t N,
                              void* y, bl_dtype ydt, int32_t* y_int, void* stream);
 
-/* The path bitlinear_forward would pick for these sizes and pointers. */
+/* The path bitlinear_forward would pick for these sizes and pointers on the
+ * current device (without a usable device, as if the register-resident
+ * kernel for 5..8 tokens were unavailable). */
 bl_path bitlinear_select_path(int64_t M, int64_t K, int64_t N,
                               const void* xq, const void* packed, const void* y,
                               const void* y_int);

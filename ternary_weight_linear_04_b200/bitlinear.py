@@ -188,7 +188,7 @@ def decode_reg_shape(K, N, sms=None):
 
 
 def decode_regm_shape(M, K, N, sms=None):
-    """Shape of the register-resident kernel for 2..4 tokens with x~ given,
+    """Shape of the register-resident kernel for 2..8 tokens with x~ given,
     as a dict, or None when that kernel does not take (M, K, N).  sms
     defaults to the current device's SM count."""
     if sms is None:
@@ -202,7 +202,7 @@ def decode_regm_shape(M, K, N, sms=None):
 
 
 def set_decode_reg(enable=True):
-    """Turn the register-resident kernels (one token fused; 2..4 tokens with
+    """Turn the register-resident kernels (one token fused; 2..8 tokens with
     x~ given) on (default) or off for later launches in this process (off:
     the shared-memory decode kernel)."""
     check(_lib.lib().bitlinear_set_decode_reg(1 if enable else 0), "bitlinear_set_decode_reg")

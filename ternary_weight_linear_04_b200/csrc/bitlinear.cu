@@ -228,7 +228,7 @@ inline bool rb_allowed(int MT, int RB) { return RB * MT <= 16; }
 // Shape forced by bitlinear_set_decode_shape (0 = chosen by the model).
 std::atomic<int> g_force_G{0}, g_force_RB{0};
 // bitlinear_set_decode_reg: 0 turns the register-resident kernels off (one
-// token fused with the quantiser; 2..4 tokens with x~ given).
+// token fused with the quantiser; 2..8 tokens with x~ given).
 std::atomic<int> g_decode_reg{1};
 
 bool decode_geometry(int MT, int64_t M, int64_t K, int64_t N, int sms, int64_t xelem,
@@ -457,12 +457,12 @@ bl_status launch_decode_reg(const bl::RegDecodeArgs& a, const RegGeom& g, cudaSt
   return BL_ERR_UNSUPPORTED;
 }
 
-// Register-resident kernel for 2..4 tokens with x~ given (decode_reg.cuh):
+// Register-resident kernel for 2..8 tokens with x~ given (decode_reg.cuh):
 // the rows of the one-token geometry (one CTA per SM, RB rows per warp), MT
-// = 2 or 4 token slots, and the smallest instantiated word count NJ that
-// covers K.  The instantiated (MT, RB, NJ) keep weights, RB * MT
-// accumulators and two activation slots within 64 registers with no spills
-// (ptxas), which leaves room for two CTAs per SM.
+// = 2, 4 or 8 token slots (RB * MT <= 32), and the smallest instantiated
+// word count NJ that covers K.  The instantiated (MT, RB, NJ) keep weights,
+// RB * MT accumulators and two activation slots in registers with no spills
+// (ptxas).
 struct RegMGeom {
   int MT = 0, RB = 0, NJ = 0, rows_per_cta = 0, grid = 0;
 };
@@ -475,8 +475,8 @@ bool regm_geometry(int64_t M, int64_t K, int64_t N, int sms, RegMGeom* g) {
   if (M < 2 || M > bl::kRegMultiMaxMT) return false;
   RegGeom g1;
   if (!reg_decode_geometry(K, N, sms, &g1)) return false;
-  const int MT = M <= 2 ? 2 : 4;
-  if (g1.RB * MT > 16) return false;
+  const int MT = M <= 2 ? 2 : (M <= 4 ? 4 : 8);
+  if (g1.RB * MT > 32) return false;
   const int64_t need = (K / 16 + 31) / 32;
   const int* list = g1.RB == 1 ? kRegMNJ1 : (g1.RB == 2 ? kRegMNJ2 : kRegMNJ4);
   const int n = g1.RB == 1 ? 7 : (g1.RB == 2 ? 6 : 4);
@@ -512,6 +512,7 @@ bl_status launch_decode_regm(const bl::RegMultiArgs& a, const RegMGeom& g, cudaS
   BL_REGM_CASE(T, 4, 2) BL_REGM_CASE(T, 4, 4) BL_REGM_CASE(T, 4, 7) BL_REGM_CASE(T, 4, 8)
   BL_REGM_MT(2)
   BL_REGM_MT(4)
+  BL_REGM_MT(8)
 #undef BL_REGM_MT
 #undef BL_REGM_CASE
   return BL_ERR_UNSUPPORTED;
@@ -618,10 +619,16 @@ bool fast_layout_ok(int64_t K, const void* xq, const void* packed, const void* y
          (y_int == nullptr || aligned(y_int, 16));
 }
 
-bl_path select_path(int64_t M, int64_t K, const void* xq, const void* packed, const void* y,
-                    const void* y_int) {
+// sms < 1: the device is unknown (the register kernel is not considered).
+bl_path select_path(int64_t M, int64_t K, int64_t N, int sms, const void* xq, const void* packed,
+                    const void* y, const void* y_int) {
   if (!fast_layout_ok(K, xq, packed, y, y_int) || K > (1 << 30)) return BL_PATH_GENERIC;
   if (decode_ok(M, K)) return BL_PATH_GEMV;
+  RegMGeom mg;
+  if (sms >= 1 && M <= bl::kRegMultiMaxMT && g_decode_reg.load(std::memory_order_relaxed) != 0 &&
+      g_force_G.load(std::memory_order_relaxed) == 0 &&
+      g_force_RB.load(std::memory_order_relaxed) == 0 && regm_geometry(M, K, N, sms, &mg))
+    return BL_PATH_GEMV;  // 5..8 tokens: the register-resident kernel
   return BL_PATH_TCGEN05;
 }
 
@@ -641,14 +648,13 @@ bl_status forward_impl(const int8_t* xq, const float* eta, const int32_t* xsum, 
   int sms = 148;
   bl_status st = device_info(&sms);
   if (st != BL_OK) return st;
-  if (path == BL_PATH_AUTO) path = select_path(M, K, xq, packed, y, y_int);
+  if (path == BL_PATH_AUTO) path = select_path(M, K, N, sms, xq, packed, y, y_int);
   const cudaStream_t s = as_stream(stream);
   if (path == BL_PATH_GEMV) {
-    if (!fast_layout_ok(K, xq, packed, y, y_int) || !decode_ok(M, K) ||
-        N > INT32_MAX / 2)
-      return BL_ERR_UNSUPPORTED;
-    // 2..4 tokens: the register-resident kernel when the CTA's share fits
-    // (and no shape is forced for the shared-memory kernel).
+    if (!fast_layout_ok(K, xq, packed, y, y_int) || N > INT32_MAX / 2) return BL_ERR_UNSUPPORTED;
+    // 2..8 tokens: the register-resident kernel when the CTA's share fits
+    // (and no shape is forced for the shared-memory kernel, which takes up
+    // to 4 tokens).
     RegMGeom mg;
     if (M >= 2 && g_decode_reg.load(std::memory_order_relaxed) != 0 &&
         g_force_G.load(std::memory_order_relaxed) == 0 &&
@@ -663,6 +669,7 @@ bl_status forward_impl(const int8_t* xq, const float* eta, const int32_t* xsum, 
       r.weights_static = (flags & BL_FLAG_WEIGHTS_STATIC) ? 1 : 0;
       return launch_decode_regm(r, mg, s);
     }
+    if (!decode_ok(M, K)) return BL_ERR_UNSUPPORTED;
     bl::DecodeArgs a = {};
     a.x = xq; a.eta = eta; a.xsum = xsum; a.M = (int)M; a.K = (int)K; a.N = (int)N;
     a.packed = packed; a.gamma = gamma; a.y = y; a.y_int = y_int;
@@ -1169,8 +1176,12 @@ bl_status bitlinear_linear(const void* x, bl_dtype xdt, int64_t M, int64_t K, co
 
 bl_path bitlinear_select_path(int64_t M, int64_t K, int64_t N, const void* xq, const void* packed,
                               const void* y, const void* y_int) {
-  (void)N;
-  return select_path(M, K, xq, packed, y, y_int);
+  int sms = 0;
+  if (device_info(&sms) != BL_OK) {
+    (void)cudaGetLastError();
+    sms = 0;
+  }
+  return select_path(M, K, N, sms, xq, packed, y, y_int);
 }
 
 #ifdef BL_TEST_HOOKS

@@ -239,7 +239,7 @@ __global__ void __launch_bounds__(kRegThreads + 64, 2) k_decode_reg(const RegDec
 }
 
 // ---------------------------------------------------------------------------
-// The same register-resident layout for 2 to 4 tokens whose x~, eta and
+// The same register-resident layout for 2 to 8 tokens whose x~, eta and
 // xsum are given (the quantiser ran before, or the caller passes x~):
 // [Production] "The MatMul-Free Breakthrough" and pipeline step 5 for a few
 // decode tokens at once.
@@ -252,11 +252,12 @@ __global__ void __launch_bounds__(kRegThreads + 64, 2) k_decode_reg(const RegDec
 //     four planes (w >> 2i) & 0x03030303 (code 4b + i in byte b, matching slot
 //     word i) and 8 dp4a.  The planes are recomputed per pair rather than
 //     kept, which holds the registers to weights + RB * MT accumulators + two
-//     slots (up to 90 at the instantiated shapes, no spills).  One CTA per
+//     slots (at most 128, no spills at the instantiated shapes).  One CTA per
 //     SM: in a decode layer the next launch is the quantiser's few CTAs,
 //     which fit beside it, and this kernel's weights stream while they run;
-//   * a transposed warp sum over the RB * MT values leaves each (row, token)
-//     total on one lane, which subtracts xsum, rescales and stores it.
+//   * a transposed warp sum over the RB * MT values (up to 32, one per lane)
+//     leaves each (row, token) total on one lane, which subtracts xsum,
+//     rescales and stores it.
 struct RegMultiArgs {
   const int8_t* xq;        // M x K
   const float* eta;        // M
@@ -271,13 +272,13 @@ struct RegMultiArgs {
   int weights_static;
 };
 
-constexpr int kRegMultiMaxMT = 4;
+constexpr int kRegMultiMaxMT = 8;
 
-// MT tokens (2 or 4; M <= MT), RB rows per warp (RB * MT <= 16), NJ words per
-// lane and row.  Shared memory: MT * 32 NJ slots of 16 bytes.
+// MT tokens (2, 4 or 8; M <= MT), RB rows per warp (RB * MT <= 32), NJ words
+// per lane and row.  Shared memory: MT * 32 NJ slots of 16 bytes.
 template <int MT, int RB, int NJ>
 __global__ void __launch_bounds__(kRegThreads, 1) k_decode_regm(const RegMultiArgs a) {
-  static_assert(MT == 2 || MT == 4, "2 or 4 tokens");
+  static_assert(MT == 2 || MT == 4 || MT == 8, "2, 4 or 8 tokens");
   static_assert(RB == 1 || RB == 2 || RB == 4, "RB rows per warp: 1, 2 or 4");
   constexpr int NWP = 32 * NJ;                           // slot words per token
   constexpr int XI = (MT * NWP + kRegThreads - 1) / kRegThreads;  // slots per thread

@@ -112,8 +112,8 @@ def test_register_kernel_shape_picks():
 
 
 def test_multi_token_register_kernel_shape_picks():
-    """The register-resident kernel for 2..4 tokens (x~ given): the rows of
-    the one-token geometry, 2 or 4 token slots, RB * MT <= 16, and the
+    """The register-resident kernel for 2..8 tokens (x~ given): the rows of
+    the one-token geometry, 2, 4 or 8 token slots, RB * MT <= 32, and the
     smallest instantiated word count that covers K."""
     L = _lib.lib()
 
@@ -127,19 +127,21 @@ def test_multi_token_register_kernel_shape_picks():
     assert regm(2, 3200, 8640) == (_lib.BL_OK, [2, 4, 7, 59, 147])
     assert regm(2, 8192, 1024) == (_lib.BL_OK, [2, 1, 17, 7, 147])
     assert regm(1, 3200, 8640) is None     # one token: the fused kernel
-    assert regm(5, 3200, 8640) is None     # more than 4 tokens
+    assert regm(5, 3200, 8640) == (_lib.BL_OK, [8, 4, 7, 59, 147])
+    assert regm(8, 8640, 3200) == (_lib.BL_OK, [8, 2, 17, 22, 146])
+    assert regm(9, 3200, 8640) is None     # more than 8 tokens
     assert regm(4, 8192, 28672) is None    # 194 rows per CTA
     assert regm(4, 3232, 100) is None      # K not a multiple of 64
     buf = (ctypes.c_int32 * 5)()
     assert L.bitlinear_decode_regm_shape(4, 3200, 8640, 0, buf) == _lib.BL_ERR_INVALID_ARG
     assert L.bitlinear_decode_regm_shape(4, 3200, 8640, 148, None) == _lib.BL_ERR_INVALID_ARG
-    for M in (2, 3, 4):
+    for M in (2, 3, 4, 5, 8):
         for K in range(64, 16384 + 1, 64):
             for N in (1, 148, 2368, 2369, 4736, 9472, 9473):
                 r = regm(M, K, N)
                 if r is None:
                     continue
                 mt, rb, nj, rpc, grid = r[1]
-                assert mt == (2 if M == 2 else 4) and rb in (1, 2, 4) and rb * mt <= 16
+                assert mt == (2 if M == 2 else (4 if M <= 4 else 8)) and rb in (1, 2, 4) and rb * mt <= 32
                 assert nj in {1: (2, 4, 7, 8, 12, 17, 24), 2: (2, 4, 7, 8, 12, 17), 4: (2, 4, 7, 8)}[rb]
                 assert rpc <= 16 * rb and 512 * nj >= K and rpc * grid >= N and (grid - 1) * rpc < N
