@@ -1085,18 +1085,36 @@ bl_status bitlinear_quant_act(const void* x, bl_dtype xdt, int64_t M, int64_t K,
   const cudaStream_t s = as_stream(stream);
   int64_t ctas = M;
   if (ctas > static_cast<int64_t>(sms) * 64) ctas = static_cast<int64_t>(sms) * 64;
+  // A few rows (decode): 1024 threads per row, the whole row in registers
+  // for K <= 16384, one read; many rows: 256 threads per row.
+  const bool wide = M <= 64;
+  const dim3 grid(static_cast<unsigned>(ctas));
   if (xdt == BL_BF16) {
     const int vec = (K % 8 == 0) && aligned(x, 16) && aligned(xq, 8);
+    const auto* xb = static_cast<const __nv_bfloat16*>(x);
+    if (wide) {
+      static int done_w[kMaxDevices] = {0};
+      if (!ensure_smem(bl::k_quant_act<__nv_bfloat16, 1024>, 0, done_w)) return BL_ERR_CUDA;
+      return launch_pdl(bl::k_quant_act<__nv_bfloat16, 1024>, grid, dim3(1024), 0, s, xb, M, K, vec, xq,
+                        eta, xsum);
+    }
     static int carve_done[kMaxDevices] = {0};
-    if (!ensure_smem(bl::k_quant_act<__nv_bfloat16>, 0, carve_done)) return BL_ERR_CUDA;
-    return launch_pdl(bl::k_quant_act<__nv_bfloat16>, dim3(static_cast<unsigned>(ctas)), dim3(256),
-                      0, s, static_cast<const __nv_bfloat16*>(x), M, K, vec, xq, eta, xsum);
+    if (!ensure_smem(bl::k_quant_act<__nv_bfloat16, 256>, 0, carve_done)) return BL_ERR_CUDA;
+    return launch_pdl(bl::k_quant_act<__nv_bfloat16, 256>, grid, dim3(256), 0, s, xb, M, K, vec, xq,
+                      eta, xsum);
   }
   const int vec = (K % 4 == 0) && aligned(x, 16) && aligned(xq, 4);
+  const auto* xf = static_cast<const float*>(x);
+  if (wide) {
+    static int done_wf[kMaxDevices] = {0};
+    if (!ensure_smem(bl::k_quant_act<float, 1024>, 0, done_wf)) return BL_ERR_CUDA;
+    return launch_pdl(bl::k_quant_act<float, 1024>, grid, dim3(1024), 0, s, xf, M, K, vec, xq, eta,
+                      xsum);
+  }
   static int carve_done_f[kMaxDevices] = {0};
-  if (!ensure_smem(bl::k_quant_act<float>, 0, carve_done_f)) return BL_ERR_CUDA;
-  return launch_pdl(bl::k_quant_act<float>, dim3(static_cast<unsigned>(ctas)), dim3(256), 0, s,
-                    static_cast<const float*>(x), M, K, vec, xq, eta, xsum);
+  if (!ensure_smem(bl::k_quant_act<float, 256>, 0, carve_done_f)) return BL_ERR_CUDA;
+  return launch_pdl(bl::k_quant_act<float, 256>, grid, dim3(256), 0, s, xf, M, K, vec, xq, eta,
+                    xsum);
 }
 
 bl_status bitlinear_forward(const int8_t* xq, const float* eta, const int32_t* xsum, int64_t M,

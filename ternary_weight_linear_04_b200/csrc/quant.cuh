@@ -196,31 +196,41 @@ __device__ __forceinline__ uint32_t pack_lowbytes(uint32_t a, uint32_t b, uint32
   return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
 }
 
-// Block-wide reductions over 256 threads.
-__device__ __forceinline__ float block_max_256(float v, float* red) {
+// Block-wide reductions over NT threads (NT a multiple of 32, at most 1024;
+// red holds NT / 32 values).
+template <int NT>
+__device__ __forceinline__ float block_max_nt(float v, float* red) {
+  static_assert(NT % 32 == 0 && NT <= 1024, "whole warps, at most 32");
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
   const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
   __syncthreads();
   if (l == 0) red[w] = v;
   __syncthreads();
-  v = (l < 8) ? red[l] : 0.0f;
+  v = (l < NT / 32) ? red[l] : 0.0f;
 #pragma unroll
-  for (int o = 4; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
-  return __shfl_sync(0xFFFFFFFFu, v, 0);
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+  return v;
 }
 
-__device__ __forceinline__ int32_t block_sum_256(int32_t v, int32_t* red) {
+template <int NT>
+__device__ __forceinline__ int32_t block_sum_nt(int32_t v, int32_t* red) {
+  static_assert(NT % 32 == 0 && NT <= 1024, "whole warps, at most 32");
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
   const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
   __syncthreads();
   if (l == 0) red[w] = v;
   __syncthreads();
-  v = (l < 8) ? red[l] : 0;
+  v = (l < NT / 32) ? red[l] : 0;
 #pragma unroll
-  for (int o = 4; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
-  return __shfl_sync(0xFFFFFFFFu, v, 0);
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ float block_max_256(float v, float* red) { return block_max_nt<256>(v, red); }
+__device__ __forceinline__ int32_t block_sum_256(int32_t v, int32_t* red) {
+  return block_sum_nt<256>(v, red);
 }
 
 // 8 activations per 16-byte load for bf16, 4 for fp32.
@@ -258,19 +268,22 @@ struct QVec<float> {
   }
 };
 
-// One 256-thread CTA per token row.  `vec` = the row can be read with
-// 16-byte loads (K a multiple of the vector width, x 16-byte aligned) and
-// xq written with 8/4-byte stores.  The first kCache vectors of each thread
-// stay in registers between the absmax pass and the quantise pass (all of
-// the row for K up to 256 * 8 * kCache bf16 values), so the row is read
-// from memory once; longer rows read the rest again.
-template <typename T>
-__global__ void __launch_bounds__(256) k_quant_act(const T* __restrict__ x, int64_t M, int64_t K,
-                                                    int vec, int8_t* __restrict__ xq,
-                                                    float* __restrict__ eta_out,
-                                                    int32_t* __restrict__ xsum_out) {
-  __shared__ float redf[8];
-  __shared__ int32_t redi[8];
+// One NT-thread CTA per token row (NT = 256 for many rows; 1024 for a few
+// rows, where the launch is latency: then the 16 values per thread kept in
+// registers cover rows up to 16384 bf16 values, and nothing is read twice).
+// `vec` = the row can be read with 16-byte loads (K a multiple of the
+// vector width, x 16-byte aligned) and xq written with 8/4-byte stores.  The
+// first kCache vectors of each thread stay in registers between the absmax
+// pass and the quantise pass (all of the row for K up to NT * 8 * kCache
+// bf16 values), so the row is read from memory once; longer rows read the
+// rest again.
+template <typename T, int NT>
+__global__ void __launch_bounds__(NT) k_quant_act(const T* __restrict__ x, int64_t M, int64_t K,
+                                                   int vec, int8_t* __restrict__ xq,
+                                                   float* __restrict__ eta_out,
+                                                   int32_t* __restrict__ xsum_out) {
+  __shared__ float redf[NT / 32];
+  __shared__ int32_t redi[NT / 32];
   constexpr int V = QVec<T>::kN;
   constexpr int kCache = 16 / V;  // 16 values per thread kept in registers
   constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
@@ -284,23 +297,23 @@ __global__ void __launch_bounds__(256) k_quant_act(const T* __restrict__ x, int6
     if (vec) {
 #pragma unroll
       for (int c = 0; c < kCache; ++c) {
-        const int64_t k = (static_cast<int64_t>(threadIdx.x) + 256 * c) * V;
+        const int64_t k = (static_cast<int64_t>(threadIdx.x) + NT * c) * V;
         if (k < K) {
           QVec<T>::load(row + k, cache[c]);
 #pragma unroll
           for (int i = 0; i < V; ++i) amax = fmaxf(amax, fabsf(cache[c][i]));
         }
       }
-      for (int64_t k = (static_cast<int64_t>(threadIdx.x) + 256 * kCache) * V; k < K; k += 256 * V) {
+      for (int64_t k = (static_cast<int64_t>(threadIdx.x) + NT * kCache) * V; k < K; k += NT * V) {
         float f[V];
         QVec<T>::load(row + k, f);
 #pragma unroll
         for (int i = 0; i < V; ++i) amax = fmaxf(amax, fabsf(f[i]));
       }
     } else {
-      for (int64_t k = threadIdx.x; k < K; k += 256) amax = fmaxf(amax, fabsf(load_as_f32(row + k)));
+      for (int64_t k = threadIdx.x; k < K; k += NT) amax = fmaxf(amax, fabsf(load_as_f32(row + k)));
     }
-    amax = block_max_256(amax, redf);
+    amax = block_max_nt<NT>(amax, redf);
     const float eta = fmaxf(amax, 1e-5f);
     const float qs = kBf16 ? 0.0f : quant_scale(eta);
     const float rr = kBf16 ? rcp_approx(eta) : 0.0f;
@@ -320,23 +333,23 @@ __global__ void __launch_bounds__(256) k_quant_act(const T* __restrict__ x, int6
     if (vec) {
 #pragma unroll
       for (int c = 0; c < kCache; ++c) {
-        const int64_t k = (static_cast<int64_t>(threadIdx.x) + 256 * c) * V;
+        const int64_t k = (static_cast<int64_t>(threadIdx.x) + NT * c) * V;
         if (k < K) quant_store(k, cache[c]);
       }
-      for (int64_t k = (static_cast<int64_t>(threadIdx.x) + 256 * kCache) * V; k < K; k += 256 * V) {
+      for (int64_t k = (static_cast<int64_t>(threadIdx.x) + NT * kCache) * V; k < K; k += NT * V) {
         float f[V];
         QVec<T>::load(row + k, f);
         quant_store(k, f);
       }
     } else {
-      for (int64_t k = threadIdx.x; k < K; k += 256) {
+      for (int64_t k = threadIdx.x; k < K; k += NT) {
         const float xv = load_as_f32(row + k);
         const int32_t q = kBf16 ? quantise_bf16(xv, eta, heta, rs, rr, eta_bf16) : quantise_fast(xv, eta, qs);
         sum += q;
         qrow[k] = static_cast<int8_t>(q);
       }
     }
-    sum = block_sum_256(sum, redi);
+    sum = block_sum_nt<NT>(sum, redi);
     if (threadIdx.x == 0) {
       eta_out[m] = eta;
       xsum_out[m] = sum;
