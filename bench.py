@@ -367,14 +367,39 @@ def load_traffic(kernel):
 
 
 def run_e2e(args, mats, M, stream, world):
-    """Through the public Python API, host buffers in, host buffers out."""
+    """Through the public Python API, host buffers in, host buffers out.
+
+    Each step copies that step's x from pinned host memory to the device,
+    runs bitlinear.linear on both matrices and copies y back to pinned host
+    memory, then synchronises the stream.  As a decode loop runs it, the
+    step's calls are captured once in a CUDA graph per rotated weight copy
+    and replayed; the same step issued eagerly from Python is timed too
+    ("eager")."""
     from ternary_weight_linear_04_b200 import bitlinear as bl
     xs_h = [m["x"].cpu().pin_memory() for m in mats]
     ys_h = [torch.empty_like(m["y"], device="cpu").pin_memory() for m in mats]
+    # The graph's step: every matrix's x in one pinned staging buffer, one
+    # copy in; every y into one device buffer, one copy out.
+    x_sizes = [m["x"].numel() for m in mats]
+    y_sizes = [m["y"].numel() for m in mats]
+    xcat_h = torch.cat([x.flatten() for x in xs_h]).pin_memory()
+    ycat_h = torch.empty(sum(y_sizes), dtype=mats[0]["y"].dtype).pin_memory()
+    xcat_d = torch.empty_like(xcat_h, device=mats[0]["x"].device)
+    ycat_d = torch.empty_like(ycat_h, device=mats[0]["y"].device)
+    xs_d = [v.view(m["x"].shape) for v, m in zip(torch.split(xcat_d, x_sizes), mats)]
+    ys_d = [v.view(m["y"].shape) for v, m in zip(torch.split(ycat_d, y_sizes), mats)]
     steps = max(3, min(args.steps, 500))
     copies = len(mats[0]["copies"])
 
-    def one(i):
+    def calls(i):
+        xcat_d.copy_(xcat_h, non_blocking=True)
+        for j, m in enumerate(mats):
+            pk, g = m["copies"][i % copies]
+            bl.linear(xs_d[j], pk, g, m["N"], out_dtype=torch.bfloat16, weights_static=True,
+                      stream=stream, out=ys_d[j])
+        ycat_h.copy_(ycat_d, non_blocking=True)
+
+    def eager(i):
         for j, m in enumerate(mats):
             pk, g = m["copies"][i % copies]
             xd = xs_h[j].to(m["x"].device, non_blocking=True)
@@ -384,22 +409,45 @@ def run_e2e(args, mats, M, stream, world):
         stream.synchronize()
 
     with torch.cuda.stream(stream):
+        for i in range(copies):
+            calls(i)
+        stream.synchronize()
+        graphs = []
+        for i in range(copies):
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr, stream=stream):
+                calls(i)
+            graphs.append(gr)
         for i in range(3):
-            one(i)
+            graphs[i % copies].replay()
+            stream.synchronize()
         barrier(world)
         t0 = time.perf_counter()
         for i in range(steps):
-            one(i)
+            graphs[i % copies].replay()
+            stream.synchronize()
         t = time.perf_counter() - t0
+        for i in range(3):
+            eager(i)
+        t1 = time.perf_counter()
+        for i in range(steps):
+            eager(i)
+        te = time.perf_counter() - t1
+    del graphs
     t = max_over_ranks(t, world)
+    te = max_over_ranks(te, world)
     b = sum(linear_bytes(M, m["K"], m["N"]) for m in mats)
     h2d = sum(M * m["K"] * 2 for m in mats)
     d2h = sum(M * m["N"] * 2 for m in mats)
     return {"value": round(world * b * steps / t / 1e9, 2), "unit": "GB/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "ms_per_step": round(t / steps * 1e3, 4), "steps": steps,
-            "note": "public API (bitlinear.linear) per matrix, pinned host x in, "
-                    "host y out, stream synchronised every step"}
+            "note": "public API (bitlinear.linear) per matrix; the step's inputs in one pinned "
+                    "host buffer, one copy in, the outputs copied out in one; captured in a CUDA "
+                    "graph and replayed every step; stream synchronised every step",
+            "eager": {"value": round(world * b * steps / te / 1e9, 2),
+                      "ms_per_step": round(te / steps * 1e3, 4),
+                      "note": "the same step issued from Python every time"}}
 
 
 def run_prefill(args, dev, stream, peaks, peak_src, world, l2):
@@ -846,8 +894,9 @@ def profile_kernels():
     serves (for ncu: capture the second launch of a kernel with -s 1 -c 1,
     or all of them): pack (decode_3b's 8640 x 3200 fp32 W), quantiser
     (prefill_7b's 2048 x 4096), RMSNorm + quantiser (2048 x 8640), the
-    one-token decode kernels on both decode_3b matrices, the shared-memory
-    decode kernel at M = 4, the tensor-core kernel on prefill_7b, the base-3
+    one-token decode kernel on both decode_3b matrices, the quantiser and
+    the register-resident kernel for four tokens (decode_3b K=3200 ->
+    N=8640), the tensor-core kernel on prefill_7b, the base-3
     kernel on decode_3b (K=3200 -> N=8640) and the generic kernel (M = 3,
     K = 1000, N = 300)."""
     from ternary_weight_linear_04_b200 import build as libbuild, inputs

@@ -22,9 +22,10 @@
 //     tiles of the first S stages are requested before griddepcontrol.wait,
 //     overlapping the preceding kernel;
 //   * warps 2-9 expand the packed codes (each thread: half of one row's 32
-//     bytes, i.e. 64 codes) to bytes in natural k order, directly in the
-//     128-byte swizzled K-major layout the MMA reads, then fence the
-//     generic->async proxy and arrive (one arrival per warp);
+//     bytes, i.e. 64 codes; a warp takes 16 consecutive rows) to bytes in
+//     natural k order, directly in the 128-byte swizzled K-major layout the
+//     MMA reads, then fence the generic->async proxy and arrive (one
+//     arrival per warp);
 //   * warp 1 (one thread) issues four 128 x BM x 32 MMAs and commits the
 //     stage back (one commit per stage: the MMA thread's issue rate bounds
 //     the small token tiles).
@@ -210,8 +211,12 @@ __global__ void __launch_bounds__(kTcThreads, BM <= 32 ? 2 : 1)
   } else {
     // ---------------- unpack, then epilogue (warps 2..9)
     const int u = warp - 2;            // 0..7
-    const int urow = (warp & 3) * 32 + lane;  // weight row (output feature) in the tile
-    const int uhalf = u >> 2;          // which half of the row's 32 packed bytes
+    // thread t = 32u + lane: row t / 2, half t % 2 of the row's 32 packed
+    // bytes, so a warp reads 512 contiguous bytes of the packed tile (no
+    // bank conflict), and the 16-byte stores of each quarter-warp (rows
+    // 4i..4i+3, both halves) land in eight different swizzle chunks
+    const int urow = 16 * u + (lane >> 1);  // weight row (output feature) in the tile
+    const int uhalf = lane & 1;        // which half of the row's 32 packed bytes
     const int r8 = urow & 7;
     uint8_t* a_row = sA + (urow >> 3) * 1024 + r8 * 128;
     bool ok = true;
