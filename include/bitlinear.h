@@ -261,9 +261,10 @@ bl_status bitlinear_forward(const int8_t* xq, const float* eta, const int32_t* x
  * caller.  BL_PATH_GEMV and BL_PATH_TCGEN05 return BL_ERR_UNSUPPORTED when
  * the inputs do not meet their layout needs (K % 64 == 0, 16-byte
  * alignment; for BL_PATH_GEMV also either M <= 4 and K * M' <= 131072,
- * M' = M rounded up to 1, 2 or 4, or 2 <= M <= 8 with a shape the
- * register-resident kernel takes, see bitlinear_decode_regm_shape); the
- * results of every path are identical.
+ * M' = M rounded up to 1, 2 or 4, or 2 <= M <= 16 with a shape the
+ * register-resident (2..8) or warp-MMA (9..16) kernel takes, see
+ * bitlinear_decode_regm_shape and bitlinear_decode_mma_shape
+ *); the results of every path are identical.
  * flags: 0 or BL_FLAG_WEIGHTS_STATIC.
  */
 bl_status bitlinear_forward_path(const int8_t* xq, const float* eta, const int32_t* xsum,
@@ -366,11 +367,43 @@ bl_status bitlinear_decode_reg_shape(int64_t K, int64_t N, int sms, int32_t* sha
 bl_status bitlinear_decode_regm_shape(int64_t M, int64_t K, int64_t N, int sms, int32_t* shape);
 
 /*
+ * Shape of the warp-MMA decode kernel for 9 to 16 tokens whose x~ is given
+ * (mma.sync m16n8k32 s8 with each CTA's weights in registers), for M
+ * tokens, K inputs and N outputs on a GPU with `sms` SMs (host logic only).
+ * The pages have no counterpart.  The library uses this kernel for
+ * 9 <= M <= 16 on the decode path (BL_PATH_GEMV, which BL_PATH_AUTO picks
+ * for these M when a decode kernel takes the shape) when this query
+ * succeeds, the kernel is on (bitlinear_set_decode_mma), the register-
+ * resident kernels are on and no decode shape is forced; otherwise the
+ * 2..8-token register kernel, the shared-memory decode kernel (M <= 4) or
+ * the tensor-core kernel.  shape (host, 7 int32) receives: token slots (16),
+ * row blocks of 16 per CTA RBK, K parts per block (16 / RBK),
+ * steps of 64 K per warp, rows per CTA, CTAs, dynamic shared memory bytes.
+ * Errors: BL_ERR_INVALID_ARG for shape == NULL, K < 1, N < 1 or sms < 1;
+ * BL_ERR_UNSUPPORTED when the kernel does not take (M, K, N): M outside
+ * 9..16, K not a multiple of 64, more than 64 rows per CTA, more K steps
+ * per warp than the register budget (24), or activation slots beyond the
+ * shared memory of one CTA.
+ */
+bl_status bitlinear_decode_mma_shape(int64_t M, int64_t K, int64_t N, int sms, int32_t* shape);
+
+/*
+ * Turn the warp-MMA decode kernel on (1, the default) or off (0) for every
+ * later launch in this process (off: the 2..8-token register kernel, the
+ * shared-memory decode kernel or the tensor-core kernel take those calls).
+ * Results are identical either way; this exists to compare the kernels.
+ * No counterpart on the pages.  Not synchronised with launches in flight
+ * on other host threads.
+ * Errors: BL_ERR_INVALID_ARG for values other than 0 and 1.
+ */
+bl_status bitlinear_set_decode_mma(int enable);
+
+/*
  * Turn the register-resident kernels on (1, the default) or off (0) for
  * every later launch in this process: the one-token kernel of
- * bitlinear_linear (quantiser fused) and the 2..8-token kernel of the
- * decode path (x~ given).  Off, those calls run the shared-memory decode
- * kernel.  Results are identical either way; this exists to compare the
+ * bitlinear_linear (quantiser fused), the 2..8-token kernel and the
+ * warp-MMA kernel of the decode path (x~ given).  Off, those calls run the
+ * shared-memory decode kernel (or, above 4 tokens, the tensor-core kernel).  Results are identical either way; this exists to compare the
  * kernels.  No counterpart on the pages.
  * Not synchronised with launches in flight on other host threads.
  * Errors: BL_ERR_INVALID_ARG for values other than 0 and 1.

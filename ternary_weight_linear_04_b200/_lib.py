@@ -42,6 +42,8 @@ SIGNATURES = {
     "bitlinear_decode_shape_for": (_I, [_I64, _I64, _I64, _I, _I, _P]),
     "bitlinear_decode_reg_shape": (_I, [_I64, _I64, _I, _P]),
     "bitlinear_decode_regm_shape": (_I, [_I64, _I64, _I64, _I, _P]),
+    "bitlinear_decode_mma_shape": (_I, [_I64, _I64, _I64, _I, _P]),
+    "bitlinear_set_decode_mma": (_I, [_I]),
     "bitlinear_set_decode_reg": (_I, [_I]),
     "bitlinear_set_decode_shape": (_I, [_I, _I]),
     "bitlinear_set_tc_split": (_I, [_I]),

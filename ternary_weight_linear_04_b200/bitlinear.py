@@ -201,6 +201,27 @@ def decode_regm_shape(M, K, N, sms=None):
     return dict(zip(("token_slots", "rows_per_warp", "words_per_lane", "rows_per_cta", "ctas"), list(buf)))
 
 
+def decode_mma_shape(M, K, N, sms=None):
+    """Shape of the warp-MMA decode kernel for 9..16 tokens with x~ given, as
+    a dict, or None when that kernel does not take (M, K, N).  sms defaults
+    to the current device's SM count."""
+    if sms is None:
+        sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    buf = (ctypes.c_int32 * 7)()
+    st = _lib.lib().bitlinear_decode_mma_shape(M, K, N, sms, buf)
+    if st == _lib.BL_ERR_UNSUPPORTED:
+        return None
+    check(st, "bitlinear_decode_mma_shape")
+    return dict(zip(("token_slots", "row_blocks", "k_parts", "k_steps", "rows_per_cta", "ctas",
+                     "smem_bytes"), list(buf)))
+
+
+def set_decode_mma(enable=True):
+    """Turn the warp-MMA decode kernel on (default) or off for later launches
+    in this process."""
+    check(_lib.lib().bitlinear_set_decode_mma(1 if enable else 0), "bitlinear_set_decode_mma")
+
+
 def set_decode_reg(enable=True):
     """Turn the register-resident kernels (one token fused; 2..8 tokens with
     x~ given) on (default) or off for later launches in this process (off:

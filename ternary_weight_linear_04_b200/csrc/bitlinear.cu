@@ -19,6 +19,7 @@
 #include "common.cuh"
 #include "decode.cuh"
 #include "decode_reg.cuh"
+#include "decode_mma.cuh"
 #include "base3.cuh"
 #include "gemm_tc.cuh"
 #include "gemv.cuh"
@@ -518,6 +519,69 @@ bl_status launch_decode_regm(const bl::RegMultiArgs& a, const RegMGeom& g, cudaS
   return BL_ERR_UNSUPPORTED;
 }
 
+// Warp-MMA decode kernel for 9..16 tokens with x~ given (decode_mma.cuh):
+// the rows of the one-token geometry (one CTA per SM), RBK blocks of 16
+// rows, KP = 16 / RBK parts of K per block, NS steps of 64 K per warp (the
+// smallest instantiated value that covers K), 8, 16 or 32 token slots, and
+// the activation slots plus partial tiles within the shared memory of one CTA.
+struct MmaGeom {
+  int NT8 = 0, RBK = 0, NS = 0, rows_per_cta = 0, grid = 0;
+  size_t smem = 0;
+};
+
+constexpr int kMmaNS[] = {4, 9, 13, 17, 24};
+std::atomic<int> g_decode_mma{1};  // bitlinear_set_decode_mma
+
+bool mma_geometry(int64_t M, int64_t K, int64_t N, int sms, MmaGeom* g) {
+  if (M <= bl::kRegMultiMaxMT || M > bl::kMmaMaxTokens) return false;
+  if (K < 64 || K % 64 != 0 || N < 1 || N > INT32_MAX / 2 || sms < 1) return false;
+  // one CTA per SM, the rows split evenly (at most 64 per CTA)
+  int64_t grid = N < sms ? N : sms;
+  const int64_t rpc = (N + grid - 1) / grid;
+  grid = (N + rpc - 1) / rpc;
+  if (rpc > 64) return false;
+  RegGeom g1;
+  g1.rows_per_cta = static_cast<int>(rpc);
+  g1.grid = static_cast<int>(grid);
+  const int rbk = g1.rows_per_cta <= 16 ? 1 : (g1.rows_per_cta <= 32 ? 2 : 4);
+  const int64_t need = (K / 64 + (16 / rbk) - 1) / (16 / rbk);
+  int ns = 0;
+  for (int v : kMmaNS)
+    if (!ns && v >= need) ns = v;
+  if (!ns) return false;
+  const int nt8 = 2;
+  const size_t smem = bl::mma_decode_smem(nt8, rbk, static_cast<int>(K));
+  if (smem + 1024 > kDecMaxSmem) return false;
+  g->NT8 = nt8;
+  g->RBK = rbk;
+  g->NS = ns;
+  g->rows_per_cta = g1.rows_per_cta;
+  g->grid = g1.grid;
+  g->smem = smem;
+  return true;
+}
+
+template <int NT8, int RBK, int NS>
+bl_status launch_decode_mma_ns(const bl::MmaDecodeArgs& a, const MmaGeom& g, cudaStream_t st) {
+  static int done[kMaxDevices] = {0};
+  auto kern = bl::k_decode_mma<NT8, RBK, NS>;
+  if (!ensure_smem(kern, g.smem, done)) return BL_ERR_CUDA;
+  return launch_pdl(kern, dim3(static_cast<unsigned>(g.grid)), dim3(bl::kMmaThreads), g.smem, st, a);
+}
+
+bl_status launch_decode_mma(const bl::MmaDecodeArgs& a, const MmaGeom& g, cudaStream_t st) {
+#define BL_MMA_CASE(T, R, S) \
+  if (g.NT8 == T && g.RBK == R && g.NS == S) return launch_decode_mma_ns<T, R, S>(a, g, st);
+#define BL_MMA_R(T, R) \
+  BL_MMA_CASE(T, R, 4) BL_MMA_CASE(T, R, 9) BL_MMA_CASE(T, R, 13) BL_MMA_CASE(T, R, 17) BL_MMA_CASE(T, R, 24)
+#define BL_MMA_T(T) BL_MMA_R(T, 1) BL_MMA_R(T, 2) BL_MMA_R(T, 4)
+  BL_MMA_T(2)
+#undef BL_MMA_T
+#undef BL_MMA_R
+#undef BL_MMA_CASE
+  return BL_ERR_UNSUPPORTED;
+}
+
 template <typename OutT>
 bl_status launch_generic(const int8_t* xq, const float* eta, int64_t M, int64_t K,
                          const uint8_t* packed, const float* gamma, int64_t N, void* y,
@@ -624,11 +688,16 @@ bl_path select_path(int64_t M, int64_t K, int64_t N, int sms, const void* xq, co
                     const void* y, const void* y_int) {
   if (!fast_layout_ok(K, xq, packed, y, y_int) || K > (1 << 30)) return BL_PATH_GENERIC;
   if (decode_ok(M, K)) return BL_PATH_GEMV;
-  RegMGeom mg;
-  if (sms >= 1 && M <= bl::kRegMultiMaxMT && g_decode_reg.load(std::memory_order_relaxed) != 0 &&
+  if (sms >= 1 && g_decode_reg.load(std::memory_order_relaxed) != 0 &&
       g_force_G.load(std::memory_order_relaxed) == 0 &&
-      g_force_RB.load(std::memory_order_relaxed) == 0 && regm_geometry(M, K, N, sms, &mg))
-    return BL_PATH_GEMV;  // 5..8 tokens: the register-resident kernel
+      g_force_RB.load(std::memory_order_relaxed) == 0) {
+    MmaGeom gm;
+    if (g_decode_mma.load(std::memory_order_relaxed) != 0 && mma_geometry(M, K, N, sms, &gm))
+      return BL_PATH_GEMV;  // 9..16 tokens: the warp-MMA kernel
+    RegMGeom mg;
+    if (M <= bl::kRegMultiMaxMT && regm_geometry(M, K, N, sms, &mg))
+      return BL_PATH_GEMV;  // 5..8 tokens: the register-resident kernel
+  }
   return BL_PATH_TCGEN05;
 }
 
@@ -655,10 +724,23 @@ bl_status forward_impl(const int8_t* xq, const float* eta, const int32_t* xsum, 
     // 2..8 tokens: the register-resident kernel when the CTA's share fits
     // (and no shape is forced for the shared-memory kernel, which takes up
     // to 4 tokens).
+    const bool reg_on = M >= 2 && g_decode_reg.load(std::memory_order_relaxed) != 0 &&
+                        g_force_G.load(std::memory_order_relaxed) == 0 &&
+                        g_force_RB.load(std::memory_order_relaxed) == 0;
+    MmaGeom gm;
+    if (reg_on && g_decode_mma.load(std::memory_order_relaxed) != 0 && mma_geometry(M, K, N, sms, &gm)) {
+      bl::MmaDecodeArgs r = {};
+      r.xq = xq; r.eta = eta; r.xsum = xsum;
+      r.M = static_cast<int>(M); r.K = static_cast<int>(K); r.N = static_cast<int>(N);
+      r.packed = packed; r.gamma = gamma; r.y = y;
+      r.y_bf16 = ydt == BL_BF16 ? 1 : 0;
+      r.y_int = y_int;
+      r.rows_per_cta = gm.rows_per_cta;
+      r.weights_static = (flags & BL_FLAG_WEIGHTS_STATIC) ? 1 : 0;
+      return launch_decode_mma(r, gm, s);
+    }
     RegMGeom mg;
-    if (M >= 2 && g_decode_reg.load(std::memory_order_relaxed) != 0 &&
-        g_force_G.load(std::memory_order_relaxed) == 0 &&
-        g_force_RB.load(std::memory_order_relaxed) == 0 && regm_geometry(M, K, N, sms, &mg)) {
+    if (reg_on && regm_geometry(M, K, N, sms, &mg)) {
       bl::RegMultiArgs r = {};
       r.xq = xq; r.eta = eta; r.xsum = xsum;
       r.M = static_cast<int>(M); r.K = static_cast<int>(K); r.N = static_cast<int>(N);
@@ -785,6 +867,26 @@ bl_status bitlinear_decode_shape(int64_t M, int64_t K, int64_t N, int fused, int
   shape[7] = g.stages;
   shape[8] = g.x_staged;
   shape[9] = static_cast<int32_t>(g.smem);
+  return BL_OK;
+}
+
+bl_status bitlinear_decode_mma_shape(int64_t M, int64_t K, int64_t N, int sms, int32_t* shape) {
+  if (!shape || K < 1 || N < 1 || sms < 1) return BL_ERR_INVALID_ARG;
+  MmaGeom g;
+  if (!mma_geometry(M, K, N, sms, &g)) return BL_ERR_UNSUPPORTED;
+  shape[0] = 8 * g.NT8;
+  shape[1] = g.RBK;
+  shape[2] = 16 / g.RBK;
+  shape[3] = g.NS;
+  shape[4] = g.rows_per_cta;
+  shape[5] = g.grid;
+  shape[6] = static_cast<int32_t>(g.smem);
+  return BL_OK;
+}
+
+bl_status bitlinear_set_decode_mma(int enable) {
+  if (enable != 0 && enable != 1) return BL_ERR_INVALID_ARG;
+  g_decode_mma.store(enable, std::memory_order_relaxed);
   return BL_OK;
 }
 

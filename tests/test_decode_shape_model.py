@@ -145,3 +145,40 @@ def test_multi_token_register_kernel_shape_picks():
                 assert mt == (2 if M == 2 else (4 if M <= 4 else 8)) and rb in (1, 2, 4) and rb * mt <= 32
                 assert nj in {1: (2, 4, 7, 8, 12, 17, 24), 2: (2, 4, 7, 8, 12, 17), 4: (2, 4, 7, 8)}[rb]
                 assert rpc <= 16 * rb and 512 * nj >= K and rpc * grid >= N and (grid - 1) * rpc < N
+
+
+def test_warp_mma_kernel_shape_picks():
+    """The warp-MMA decode kernel for 9..16 tokens (x~ given): the rows of the
+    one-token geometry, blocks of 16 rows (RBK), 16 / RBK parts of K, the
+    smallest instantiated step count covering K, 16 token slots, and
+    the activation slots plus partial tiles within one CTA's shared memory;
+    up to 8 tokens the register kernel runs instead."""
+    L = _lib.lib()
+
+    def mma(M, K, N, sms=148):
+        buf = (ctypes.c_int32 * 7)()
+        st = L.bitlinear_decode_mma_shape(M, K, N, sms, buf)
+        return None if st == _lib.BL_ERR_UNSUPPORTED else (st, list(buf))
+
+    assert mma(16, 3200, 8640) == (_lib.BL_OK, [16, 4, 4, 13, 59, 147, 68608])
+    assert mma(16, 8640, 3200) == (_lib.BL_OK, [16, 2, 8, 17, 22, 146, 154624])
+    assert mma(9, 3200, 8640) == (_lib.BL_OK, [16, 4, 4, 13, 59, 147, 68608])
+    assert mma(8, 3200, 8640) is None       # 8 tokens: the register kernel
+    assert mma(17, 3200, 8640) is None      # more than 16 tokens: the tensor-core kernel
+    assert mma(16, 8192, 8192) is None      # 32 steps per warp: beyond the register budget
+    assert mma(16, 8192, 28672) is None     # 194 rows per CTA
+    assert mma(12, 3232, 100) is None       # K not a multiple of 64
+    buf = (ctypes.c_int32 * 7)()
+    assert L.bitlinear_decode_mma_shape(12, 3200, 8640, 0, buf) == _lib.BL_ERR_INVALID_ARG
+    assert L.bitlinear_decode_mma_shape(12, 3200, 8640, 148, None) == _lib.BL_ERR_INVALID_ARG
+    assert L.bitlinear_set_decode_mma(2) == _lib.BL_ERR_INVALID_ARG
+    for M in (9, 12, 16):
+        for K in range(64, 24576 + 1, 64):
+            for N in (1, 148, 2368, 2369, 4736, 9472, 9473):
+                r = mma(M, K, N)
+                if r is None:
+                    continue
+                slots, rbk, kp, ns, rpc, grid, smem = r[1]
+                assert slots == 16 and rbk * kp == 16
+                assert ns in (4, 9, 13, 17, 24) and kp * ns * 64 >= K and rpc <= 16 * rbk
+                assert rpc * grid >= N and (grid - 1) * rpc < N and smem + 1024 <= 227 * 1024

@@ -754,3 +754,69 @@ def test_multi_token_linear_uses_quantiser_then_register_kernel(M, K, N):
     np.testing.assert_array_equal(xsum.cpu().numpy(), ref_xsum)
     np.testing.assert_array_equal(y_int.cpu().numpy(), ref_yint)
     np.testing.assert_array_equal(y_bits(y.cpu()), orc.f32_to_bf16_bits(ref_y))
+
+
+# ----------------------------------------------------------------- 2..32 tokens, warp-level MMA
+
+_MMA_CASES = ([(K, 8640) for K in (1024, 2048, 3200, 4096, 6144)]
+              + [(K, 3200) for K in (2048, 4096, 6144, 8640, 12288)]
+              + [(K, 1000) for K in (4096, 8192, 12288, 16384, 24576)]
+              + [(64, 5), (3200, 8641), (8640, 2369), (1024, 149)])
+
+
+@pytest.fixture
+def mma_kernel():
+    yield bl.set_decode_mma
+    bl.set_decode_mma(True)
+
+
+@pytest.mark.parametrize("M", [9, 12, 16])
+@pytest.mark.parametrize("K,N", _MMA_CASES)
+def test_warp_mma_decode_kernel_every_shape(mma_kernel, M, K, N):
+    """bitlinear_forward (x~ given) for 9..16 tokens on the warp-MMA kernel:
+    every (token slots, row blocks, K steps) instantiation, ragged last CTAs
+    and row blocks, padding words, tokens and K steps, static and non-static
+    weights, fp32 and bf16 y; y_int and y bit-exact against the oracle, and
+    identical with the kernel switched off."""
+    if bl.decode_mma_shape(M, K, N) is None:
+        # the activation slots of 16 tokens fit one CTA's shared memory up to
+        # K = 12288
+        assert K > 12288, "the warp-MMA kernel takes this shape"
+        pytest.skip("the activation slots of this many tokens exceed one CTA's shared memory")
+    W, x = inputs.make_case(14000 + 11 * M + K + N, M, K, N, act_dtype="bf16")
+    ref_packed, ref_gamma, _ = orc.pack_weights(W)
+    _, _, packed, gamma = gpu_pack(W)
+    ref_xq, ref_eta, ref_xsum = orc.quant_act(x)
+    ref_yint, ref_y = orc.forward(ref_xq, ref_eta, ref_packed, ref_gamma, K, N)
+    xq, eta, xsum = (torch.from_numpy(a).cuda() for a in (ref_xq, ref_eta, ref_xsum.astype(np.int32)))
+    for static in (True, False):
+        for out in ("bf16", "f32"):
+            y, y_int = bl.forward(xq, eta, xsum, packed, gamma, N, out_dtype=DT[out], want_int=True,
+                                  path="gemv", weights_static=static)
+            np.testing.assert_array_equal(y_int.cpu().numpy(), ref_yint)
+            np.testing.assert_array_equal(y_bits(y.cpu()), oracle_y_bits(ref_y, out))
+    mma_kernel(False)
+    y_off = bl.forward(xq, eta, xsum, packed, gamma, N, out_dtype=torch.bfloat16)
+    np.testing.assert_array_equal(y_bits(y_off.cpu()), orc.f32_to_bf16_bits(ref_y))
+
+
+@pytest.mark.parametrize("M", [9, 16, 24])
+@pytest.mark.parametrize("K,N", [(3200, 8640), (8640, 3200)])
+def test_warp_mma_linear_on_decode_shapes(M, K, N):
+    """bitlinear_linear for 9..24 tokens on decode_3b's matrices (quantiser,
+    then the warp-MMA kernel up to 16 tokens, the tensor-core kernel above):
+    x~, eta, xsum, y_int and y bit-exact."""
+    W, x = inputs.make_case(14500 + M + K, M, K, N, act_dtype="bf16")
+    ref_packed, ref_gamma, _ = orc.pack_weights(W)
+    _, _, packed, gamma = gpu_pack(W)
+    ref_xq, ref_eta, ref_xsum = orc.quant_act(x)
+    ref_yint, ref_y = orc.forward(ref_xq, ref_eta, ref_packed, ref_gamma, K, N)
+    xd = torch.from_numpy(x).cuda().to(torch.bfloat16)
+    want_path = "gemv" if M <= 16 else "tcgen05"  # above 16 tokens: the tensor-core kernel
+    assert bl.select_path(M, K, N, xd, packed, xd) == want_path
+    y, (xq, eta, xsum), y_int = bl.linear(xd, packed, gamma, N, out_dtype=torch.bfloat16, want_quant=True,
+                                          want_int=True, weights_static=True)
+    np.testing.assert_array_equal(xq.cpu().numpy(), ref_xq)
+    np.testing.assert_array_equal(xsum.cpu().numpy(), ref_xsum)
+    np.testing.assert_array_equal(y_int.cpu().numpy(), ref_yint)
+    np.testing.assert_array_equal(y_bits(y.cpu()), orc.f32_to_bf16_bits(ref_y))
