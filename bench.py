@@ -894,9 +894,10 @@ def profile_kernels():
     serves (for ncu: capture the second launch of a kernel with -s 1 -c 1,
     or all of them): pack (decode_3b's 8640 x 3200 fp32 W), quantiser
     (prefill_7b's 2048 x 4096), RMSNorm + quantiser (2048 x 8640), the
-    one-token decode kernel on both decode_3b matrices, the quantiser and
-    the register-resident kernel for four tokens (decode_3b K=3200 ->
-    N=8640), the tensor-core kernel on prefill_7b, the base-3
+    one-token decode kernel on both decode_3b matrices, the quantiser with
+    the register-resident kernel for four tokens and with the warp-MMA
+    kernel for sixteen (decode_3b K=3200 -> N=8640), the tensor-core kernel
+    on prefill_7b, the base-3
     kernel on decode_3b (K=3200 -> N=8640) and the generic kernel (M = 3,
     K = 1000, N = 300)."""
     from ternary_weight_linear_04_b200 import build as libbuild, inputs
@@ -907,7 +908,7 @@ def profile_kernels():
     wl = inputs.WORKLOADS["decode_3b"]
     mats = []
     for j in range(2):
-        W, x = inputs.make_matrix_inputs(wl, j, m_max=4)
+        W, x = inputs.make_matrix_inputs(wl, j, m_max=16)
         mats.append((torch.from_numpy(W).to(dev), torch.from_numpy(x).to(dev).to(torch.bfloat16)))
     pw = inputs.WORKLOADS["prefill_7b"]
     Wp, xp = inputs.make_matrix_inputs(pw, 0)
@@ -924,6 +925,7 @@ def profile_kernels():
             bl.linear(x[:1], pk, g, W.shape[0], weights_static=True)
         pk, g = packed[0]
         bl.linear(mats[0][1][:4], pk, g, mats[0][0].shape[0], weights_static=True)
+        bl.linear(mats[0][1][:16], pk, g, mats[0][0].shape[0], weights_static=True)
         ppk, pg = bl.pack_weights(Wp)
         xq, eta, xsum = bl.quant_act(xp)
         bl.forward(xq, eta, xsum, ppk, pg, Wp.shape[0], weights_static=True)

@@ -286,18 +286,20 @@ bl_status bitlinear_forward_path(const int8_t* xq, const float* eta, const int32
  *   packed, gamma, N  in   as for bitlinear_forward.
  *   y, ydt, y_int     out  as for bitlinear_forward (y_int optional).
  *   xq, eta, xsum     out  the quantised activations (M x K int8, M fp32,
- *                          M int32).  For bf16 decode batches of one or
- *                          two tokens (M <= 2, K % 64 == 0, K * M' <=
- *                          131072 with M' = M rounded up to 1 or 2, 16-byte
- *                          aligned x, packed, y) one fused kernel runs and
- *                          these are optional (NULL = not written).  For
- *                          one token whose layer fits it (see
- *                          bitlinear_decode_reg_shape), that kernel holds
- *                          each CTA's weights in registers.
- *                          Otherwise two kernels run (quantiser, then the
- *                          accumulate kernel bitlinear_forward would pick)
- *                          and they are required scratch
- *                          (BL_ERR_INVALID_ARG if NULL).
+ *                          M int32).  For bf16 decode batches one fused
+ *                          kernel runs and these are optional (NULL = not
+ *                          written): one token whose layer fits the
+ *                          register-resident kernel (see
+ *                          bitlinear_decode_reg_shape), two tokens whose
+ *                          layer fits the multi-token one (see
+ *                          bitlinear_decode_regm_shape; 16-byte aligned x,
+ *                          packed, y, y_int and xq), and otherwise one or
+ *                          two tokens with K % 64 == 0, K * M' <= 131072
+ *                          (M' = M rounded up to 1 or 2) and 16-byte
+ *                          aligned x, packed, y.  Otherwise two kernels run
+ *                          (quantiser, then the accumulate kernel
+ *                          bitlinear_forward would pick) and they are
+ *                          required scratch (BL_ERR_INVALID_ARG if NULL).
  *   flags             in   0 or BL_FLAG_WEIGHTS_STATIC.
  */
 bl_status bitlinear_linear(const void* x, bl_dtype xdt, int64_t M, int64_t K,
@@ -349,9 +351,11 @@ bl_status bitlinear_decode_shape_for(int64_t M, int64_t K, int64_t N, int fused,
 bl_status bitlinear_decode_reg_shape(int64_t K, int64_t N, int sms, int32_t* shape);
 
 /*
- * Shape of the register-resident kernel for 2 to 8 tokens whose x~ is given
- * (BL_PATH_GEMV of bitlinear_forward, and the accumulate step of
- * bitlinear_linear from 3 tokens on), for M tokens, K inputs and N outputs
+ * Shape of the register-resident kernel for 2 to 8 tokens (BL_PATH_GEMV of
+ * bitlinear_forward with x~ given; bitlinear_linear runs it after the
+ * quantiser kernel from three tokens on, and with the quantiser fused for
+ * two bf16 tokens: every CTA quantises both rows), for M tokens, K inputs
+ * and N outputs
  * on a GPU with `sms` SMs (host logic only; usable without a GPU).  The
  * pages have no counterpart.  The library uses this kernel for 2 <= M <= 8
  * on the decode path when this query succeeds and no decode shape is forced

@@ -493,18 +493,24 @@ bool regm_geometry(int64_t M, int64_t K, int64_t N, int sms, RegMGeom* g) {
   return true;
 }
 
-template <int MT, int RB, int NJ>
+template <int MT, int RB, int NJ, bool FUSE>
 bl_status launch_decode_regm_nj(const bl::RegMultiArgs& a, const RegMGeom& g, cudaStream_t st) {
   static int done[kMaxDevices] = {0};
-  auto kern = bl::k_decode_regm<MT, RB, NJ>;
+  auto kern = bl::k_decode_regm<MT, RB, NJ, FUSE>;
   const size_t smem = static_cast<size_t>(MT) * 32 * NJ * 16;
   if (!ensure_smem(kern, smem, done)) return BL_ERR_CUDA;
   return launch_pdl(kern, dim3(static_cast<unsigned>(g.grid)), dim3(bl::kRegThreads), smem, st, a);
 }
 
-bl_status launch_decode_regm(const bl::RegMultiArgs& a, const RegMGeom& g, cudaStream_t st) {
-#define BL_REGM_CASE(T, R, J) \
-  if (g.MT == T && g.RB == R && g.NJ == J) return launch_decode_regm_nj<T, R, J>(a, g, st);
+// fuse: the CTA quantises bf16 x itself (bitlinear_linear, two tokens);
+// otherwise x~ is given.
+bl_status launch_decode_regm(const bl::RegMultiArgs& a, const RegMGeom& g, bool fuse, cudaStream_t st) {
+#define BL_REGM_CASE(T, R, J)                                                        \
+  if (g.MT == T && g.RB == R && g.NJ == J) {                                         \
+    if constexpr (T == 2)                                                            \
+      if (fuse) return launch_decode_regm_nj<T, R, J, true>(a, g, st);               \
+    return fuse ? BL_ERR_UNSUPPORTED : launch_decode_regm_nj<T, R, J, false>(a, g, st); \
+  }
 #define BL_REGM_MT(T)                                                                              \
   BL_REGM_CASE(T, 1, 2) BL_REGM_CASE(T, 1, 4) BL_REGM_CASE(T, 1, 7) BL_REGM_CASE(T, 1, 8)          \
   BL_REGM_CASE(T, 1, 12) BL_REGM_CASE(T, 1, 17) BL_REGM_CASE(T, 1, 24)                             \
@@ -749,7 +755,7 @@ bl_status forward_impl(const int8_t* xq, const float* eta, const int32_t* xsum, 
       r.y_int = y_int;
       r.rows_per_cta = mg.rows_per_cta;
       r.weights_static = (flags & BL_FLAG_WEIGHTS_STATIC) ? 1 : 0;
-      return launch_decode_regm(r, mg, s);
+      return launch_decode_regm(r, mg, false, s);
     }
     if (!decode_ok(M, K)) return BL_ERR_UNSUPPORTED;
     bl::DecodeArgs a = {};
@@ -1243,10 +1249,34 @@ bl_status bitlinear_linear(const void* x, bl_dtype xdt, int64_t M, int64_t K, co
   if (M == 0) return BL_OK;
   if (!x || !y) return BL_ERR_INVALID_ARG;
   if (127 * K >= (int64_t{1} << 31)) return BL_ERR_UNSUPPORTED;
-  // One fused kernel for one or two tokens; from three tokens on, the fused
-  // kernel's per-CTA quantiser (every CTA quantises all M rows) costs more
-  // than the separate quantiser kernel (measured: M = 4, K = 8640 fused
-  // 17.6 us against 4.5 + 8.3 us), so two kernels run.
+  // One fused launch for one or two bf16 tokens (a register-resident kernel
+  // when it takes the layer, else the shared-memory kernel); from three
+  // tokens on the quantiser kernel, then the accumulate.
+  int sms = 148;
+  // Two bf16 tokens whose layer the register kernel takes: one fused launch
+  // (every CTA quantises both rows itself), x~ / eta / xsum optional.  From
+  // three tokens on, quantising every row in every CTA costs more than the
+  // separate quantiser launch (decode_3b layer step, fused against two
+  // kernels: M = 3 17.1 / 14.7 us, M = 4 18.3 / 15.7 us, M = 8 29.4 / 20.6 us).
+  RegMGeom fmg;
+  if (M == 2 && xdt == BL_BF16 && device_info(&sms) == BL_OK &&
+      g_decode_reg.load(std::memory_order_relaxed) != 0 &&
+      g_force_G.load(std::memory_order_relaxed) == 0 &&
+      g_force_RB.load(std::memory_order_relaxed) == 0 && aligned(x, 16) && aligned(packed, 16) &&
+      aligned(y, 16) && (!y_int || aligned(y_int, 16)) && (!xq || aligned(xq, 16)) &&
+      (!eta || aligned(eta, 4)) && (!xsum || aligned(xsum, 4)) &&
+      regm_geometry(M, K, N, sms, &fmg)) {
+    bl::RegMultiArgs r = {};
+    r.x = static_cast<const __nv_bfloat16*>(x);
+    r.xq_out = xq; r.eta_out = eta; r.xsum_out = xsum;
+    r.M = static_cast<int>(M); r.K = static_cast<int>(K); r.N = static_cast<int>(N);
+    r.packed = packed; r.gamma = gamma; r.y = y;
+    r.y_bf16 = ydt == BL_BF16 ? 1 : 0;
+    r.y_int = y_int;
+    r.rows_per_cta = fmg.rows_per_cta;
+    r.weights_static = (flags & BL_FLAG_WEIGHTS_STATIC) ? 1 : 0;
+    return launch_decode_regm(r, fmg, true, as_stream(stream));
+  }
   const bool fused = M <= kFusedMaxM && decode_ok(M, K) && xdt == BL_BF16 &&
                      aligned(x, 16) && aligned(packed, 16) && aligned(y, 16) &&
                      (!y_int || aligned(y_int, 16)) && (!xq || aligned(xq, 16)) &&
@@ -1259,7 +1289,6 @@ bl_status bitlinear_linear(const void* x, bl_dtype xdt, int64_t M, int64_t K, co
     return forward_impl(xq, eta, xsum, M, K, packed, gamma, N, y, ydt, y_int, BL_PATH_AUTO, flags,
                         stream);
   }
-  int sms = 148;
   bl_status st = device_info(&sms);
   if (st != BL_OK) return st;
   const cudaStream_t s = as_stream(stream);

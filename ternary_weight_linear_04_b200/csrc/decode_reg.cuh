@@ -259,9 +259,13 @@ __global__ void __launch_bounds__(kRegThreads + 64, 2) k_decode_reg(const RegDec
 //     leaves each (row, token) total on one lane, which subtracts xsum,
 //     rescales and stores it.
 struct RegMultiArgs {
-  const int8_t* xq;        // M x K
+  const int8_t* xq;        // M x K (x~ given)
   const float* eta;        // M
   const int32_t* xsum;     // M
+  const __nv_bfloat16* x;  // M x K (fused: quantised by every CTA)
+  int8_t* xq_out;          // fused, optional: CTA 0 writes x~, eta, xsum
+  float* eta_out;
+  int32_t* xsum_out;
   int M, K, N;
   const uint8_t* packed;
   const float* gamma;
@@ -275,8 +279,10 @@ struct RegMultiArgs {
 constexpr int kRegMultiMaxMT = 8;
 
 // MT tokens (2, 4 or 8; M <= MT), RB rows per warp (RB * MT <= 32), NJ words
-// per lane and row.  Shared memory: MT * 32 NJ slots of 16 bytes.
-template <int MT, int RB, int NJ>
+// per lane and row; FUSE: the CTA quantises the bf16 rows itself (used for
+// two tokens: from three on the separate quantiser launch is cheaper).  Shared
+// memory: MT * 32 NJ slots of 16 bytes.
+template <int MT, int RB, int NJ, bool FUSE>
 __global__ void __launch_bounds__(kRegThreads, 1) k_decode_regm(const RegMultiArgs a) {
   static_assert(MT == 2 || MT == 4 || MT == 8, "2, 4 or 8 tokens");
   static_assert(RB == 1 || RB == 2 || RB == 4, "RB rows per warp: 1, 2 or 4");
@@ -317,9 +323,91 @@ __global__ void __launch_bounds__(kRegThreads, 1) k_decode_regm(const RegMultiAr
     gamma = __ldg(a.gamma);
   }
 
-  // x~ slots: slot q = m * NWP + w holds the 16 activations of word w of
-  // token m, transposed (byte b of slot word i = activation 16 w + 4 b + i).
-  {
+  if constexpr (FUSE) {
+    // The quantiser of [Production] "2. Absmax Dynamic Activation
+    // Quantization" for every row, in every CTA: G = 16 / MT warps per
+    // token; pass 1 takes max |x| (bit patterns of non-negative bf16 values
+    // order like the values), pass 2 reads the chunks again (from L1),
+    // quantises them with the division-free exact rule of code_bits_bf16_r
+    // and scatters the codes into the transposed slots; padding words and
+    // tokens stay zero.
+    constexpr int G = 16 / MT;
+    constexpr int XCF = (2 * NJ + G - 1) / G;  // 8-value chunks per thread and token (K <= 512 NJ)
+    __shared__ uint32_t s_max[16];
+    const int m = warp / G;                    // this warp's token
+    const int gt = (warp - m * G) * 32 + lane;  // thread within the token's warps
+    const int nch = K >> 3;
+    const uint4* x4 = reinterpret_cast<const uint4*>(a.x + static_cast<int64_t>(m) * K);
+    for (int i = tid; i < MT * NWP; i += kRegThreads) xslot[i] = make_uint4(0, 0, 0, 0);
+    if (tid < MT) s_xsum[tid] = 0;
+    uint32_t amax = 0;
+#pragma unroll
+    for (int i = 0; i < XCF; ++i) {
+      const int c = gt + 32 * G * i;
+      const uint4 v = (m < M && c < nch) ? x4[c] : make_uint4(0, 0, 0, 0);
+      const uint32_t w4[4] = {v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu, v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) amax = max(amax, max(w4[k] << 16, w4[k] & 0xFFFF0000u));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = max(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+    if (lane == 0) s_max[warp] = amax;
+    __syncthreads();  // also orders the zeroed slots before the scatter below
+    uint32_t e = 0;
+#pragma unroll
+    for (int i = 0; i < G; ++i) e = max(e, s_max[m * G + i]);
+    const float eta = fmaxf(__uint_as_float(e), 1e-5f);
+    const float rr = rcp_approx(eta);
+    const float qs = __fmul_rn(127.0f, rr);
+    const float heta = __fmul_rn(0.5f, eta);
+    const bool eta_bf16 = is_bf16_value(eta);  // else eta is the 1e-5 floor: exact quotients
+    const bool write_xq = a.xq_out != nullptr && blockIdx.x == 0;
+    int32_t psum = 0;
+#pragma unroll
+    for (int i = 0; i < XCF; ++i) {
+      const int c = gt + 32 * G * i;
+      if (m < M && c < nch) {
+        const uint4 v = x4[c];
+        uint32_t lo, hi;
+        if (eta_bf16) {
+          const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+          uint32_t q[8];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            q[2 * k] = code_bits_bf16_r(__uint_as_float(u[k] << 16), eta, heta, qs, rr);
+            q[2 * k + 1] = code_bits_bf16_r(__uint_as_float(u[k] & 0xFFFF0000u), eta, heta, qs, rr);
+          }
+          lo = pack_lowbytes(q[0], q[1], q[2], q[3]);
+          hi = pack_lowbytes(q[4], q[5], q[6], q[7]);
+        } else {
+          const uint2 lh = quantise_chunk_exact(v, eta);
+          lo = lh.x;
+          hi = lh.y;
+        }
+        psum = __dp4a(static_cast<int>(lo), 0x01010101, psum);
+        psum = __dp4a(static_cast<int>(hi), 0x01010101, psum);
+        if (write_xq) *reinterpret_cast<uint2*>(a.xq_out + static_cast<int64_t>(m) * K + 8 * c) = make_uint2(lo, hi);
+        // chunk c is half h = c & 1 of slot c >> 1 of token m: its bytes j
+        // (lo) and j (hi) go to slot word j, bytes 2h and 2h + 1
+        uint8_t* sl = smem + (static_cast<size_t>(m) * NWP + (c >> 1)) * 16 + 2 * (c & 1);
+        *reinterpret_cast<uint16_t*>(sl + 0) = static_cast<uint16_t>(__byte_perm(lo, hi, 0x0040));
+        *reinterpret_cast<uint16_t*>(sl + 4) = static_cast<uint16_t>(__byte_perm(lo, hi, 0x0051));
+        *reinterpret_cast<uint16_t*>(sl + 8) = static_cast<uint16_t>(__byte_perm(lo, hi, 0x0062));
+        *reinterpret_cast<uint16_t*>(sl + 12) = static_cast<uint16_t>(__byte_perm(lo, hi, 0x0073));
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) psum += __shfl_xor_sync(0xFFFFFFFFu, psum, o);
+    if (lane == 0 && m < M && psum != 0) atomicAdd(&s_xsum[m], psum);
+    if (gt == 0 && m < M) {
+      s_scale[m] = token_scale(eta, gamma);
+      if (blockIdx.x == 0 && a.eta_out) a.eta_out[m] = eta;
+    }
+    __syncthreads();
+    if (blockIdx.x == 0 && a.xsum_out && tid < M) a.xsum_out[tid] = s_xsum[tid];
+  } else {
+    // x~ slots: slot q = m * NWP + w holds the 16 activations of word w of
+    // token m, transposed (byte b of slot word i = activation 16 w + 4 b + i).
     uint4 v[XI];
 #pragma unroll
     for (int i = 0; i < XI; ++i) {
@@ -338,12 +426,13 @@ __global__ void __launch_bounds__(kRegThreads, 1) k_decode_regm(const RegMultiAr
         xslot[q] = t;
       }
     }
+    if (tid < MT) {
+      s_scale[tid] = tid < M ? token_scale(a.eta[tid], gamma) : 0.0f;
+      s_xsum[tid] = tid < M ? a.xsum[tid] : 0;
+    }
+    __syncthreads();
   }
-  if (tid < MT) {
-    s_scale[tid] = tid < M ? token_scale(a.eta[tid], gamma) : 0.0f;
-    s_xsum[tid] = tid < M ? a.xsum[tid] : 0;
-  }
-  __syncthreads();
+
   if (row0 >= nrows) return;  // whole warps
 
   constexpr int V = RB * MT;

@@ -820,3 +820,43 @@ def test_warp_mma_linear_on_decode_shapes(M, K, N):
     np.testing.assert_array_equal(xsum.cpu().numpy(), ref_xsum)
     np.testing.assert_array_equal(y_int.cpu().numpy(), ref_yint)
     np.testing.assert_array_equal(y_bits(y.cpu()), orc.f32_to_bf16_bits(ref_y))
+
+
+_REGM_FUSED_CASES = [(1024, 1000), (3200, 1000), (8640, 1000), (12288, 1000), (3200, 3200), (8640, 3200),
+                     (2048, 8640), (3200, 8640), (64, 5), (3200, 8641), (8640, 2369)]
+
+
+@pytest.mark.parametrize("M", [2, 3, 4, 5, 8])
+@pytest.mark.parametrize("K,N", _REGM_FUSED_CASES)
+def test_multi_token_fused_layer_every_shape(register_kernels, M, K, N):
+    """bitlinear_linear for 2..8 bf16 tokens on the register kernel, with the
+    quantiser fused at two tokens (every CTA quantises both rows) and the
+    quantiser kernel before it from three tokens on: every rows-per-warp
+    value, ragged last CTAs, padding words and tokens, one token whose |x|
+    are all below 1e-5 (eta is the 1e-5 floor: IEEE quotients), the optional
+    x~ / eta / xsum outputs present or not, static and non-static weights,
+    fp32 and bf16 y; bit-exact against the oracle and against the two-kernel
+    path (register kernels off)."""
+    assert bl.decode_regm_shape(M, K, N) is not None, "the register kernel takes (M, K, N)"
+    W, x = inputs.make_case(15000 + 13 * M + K + N, M, K, N, act_dtype="bf16")
+    rng = np.random.default_rng(M + K)
+    bits = rng.integers(0x3000, 0x3727, size=K).astype(np.uint32)
+    x[M - 1] = ((bits << 16).view(np.float32) * np.where(rng.random(K) < 0.5, -1, 1)).astype(np.float32)
+    ref_packed, ref_gamma, _ = orc.pack_weights(W)
+    _, _, packed, gamma = gpu_pack(W)
+    ref_xq, ref_eta, ref_xsum = orc.quant_act(x)
+    ref_yint, ref_y = orc.forward(ref_xq, ref_eta, ref_packed, ref_gamma, K, N)
+    xd = torch.from_numpy(x).cuda().to(torch.bfloat16)
+    for static in (True, False):
+        y, (xq, eta, xsum), y_int = bl.linear(xd, packed, gamma, N, out_dtype=torch.bfloat16, want_quant=True,
+                                              want_int=True, weights_static=static)
+        np.testing.assert_array_equal(xq.cpu().numpy(), ref_xq)
+        np.testing.assert_array_equal(eta.cpu().numpy().view(np.uint32), ref_eta.view(np.uint32))
+        np.testing.assert_array_equal(xsum.cpu().numpy(), ref_xsum)
+        np.testing.assert_array_equal(y_int.cpu().numpy(), ref_yint)
+        np.testing.assert_array_equal(y_bits(y.cpu()), orc.f32_to_bf16_bits(ref_y))
+    y32 = bl.linear(xd, packed, gamma, N, out_dtype=torch.float32, weights_static=True)
+    np.testing.assert_array_equal(y32.cpu().numpy().view(np.uint32), ref_y.view(np.uint32))
+    register_kernels(False)
+    y_off = bl.linear(xd, packed, gamma, N, out_dtype=torch.bfloat16, weights_static=True)
+    np.testing.assert_array_equal(y_bits(y_off.cpu()), orc.f32_to_bf16_bits(ref_y))
