@@ -612,7 +612,27 @@ def make_bench_mats(wl_name, M, dev, stream, l2, copies=None):
     return mats, copies, wbytes
 
 
-def run_sweep(mats, stream, world, peaks, Ms=(4, 8, 16, 32, 64)):
+def layer_kernels(M, m):
+    """The kernels bitlinear_linear launches for a bf16 layer of M tokens on
+    the matrix m, from the library's own shape queries."""
+    from ternary_weight_linear_04_b200 import bitlinear as bl
+    K, N = m["K"], m["N"]
+    if M == 1 and bl.decode_reg_shape(K, N) is not None:
+        return "k_decode_reg (fused)"
+    if M == 2 and bl.decode_regm_shape(M, K, N) is not None:
+        return "k_decode_regm (fused)"
+    if M <= 2 and bl.fused_decode_ok(M, K):
+        return "k_decode (fused)"
+    if M <= 8 and bl.decode_regm_shape(M, K, N) is not None:
+        return "k_quant_act + k_decode_regm"
+    if M <= 16 and bl.decode_mma_shape(M, K, N) is not None:
+        return "k_quant_act + k_decode_mma"
+    if bl.select_path(M, K, N, m["x_all"], m["packed"], m["x_all"]) == "gemv":
+        return "k_quant_act + k_decode"
+    return "k_quant_act + k_gemm_tc"
+
+
+def run_sweep(mats, stream, world, peaks, Ms=(2, 4, 8, 12, 16, 32, 64)):
     """decode_3b at the other batch sizes: GB/s against HBM."""
     from ternary_weight_linear_04_b200 import bitlinear as bl
     hbm = float(peaks["hbm_gbs"])
@@ -620,8 +640,7 @@ def run_sweep(mats, stream, world, peaks, Ms=(4, 8, 16, 32, 64)):
     for M in Ms:
         t = time_linear_step(mats, M, stream, world, xkey="x_all")
         b = sum(linear_bytes(M, m["K"], m["N"]) for m in mats)
-        paths = ["gemv (fused)" if bl.fused_decode_ok(M, m["K"]) else
-                 bl.select_path(M, m["K"], m["N"], m["x_all"], m["packed"], m["x_all"]) for m in mats]
+        paths = [layer_kernels(M, m) for m in mats]
         rows.append({"M": M, "us_per_step": round(t * 1e6, 2), "gbs": round(b / t / 1e9, 1),
                      "frac": round(b / t / 1e9 / hbm, 4), "paths": paths})
     return {"workload": "decode_3b: K=3200->N=8640 and K=8640->N=3200, bf16 in/out",
