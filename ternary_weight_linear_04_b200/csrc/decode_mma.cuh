@@ -31,9 +31,12 @@
 //   * tokens in tiles of 8 (the MMA's N); the token stride of the slots is
 //     padded to 4 mod 8 slots, so the 16-byte loads of a quarter-warp (two
 //     tokens, four words) hit eight different bank groups;
-//   * the KP partial 16 x 8 tiles of a block go through shared memory; after
-//     one barrier each thread adds the parts of one (row, token), subtracts
-//     xsum, rescales and stores.
+//   * the KP partial 16 x 8 tiles of a block go through shared memory, laid
+//     out [K part][token][CTA row] with the token stride padded to 4 mod 32
+//     words: the fragment stores of a warp fall in 32 different banks and
+//     the reads, consecutive rows of one token per warp, in consecutive
+//     banks; after one barrier each thread adds the parts of one (row,
+//     token), subtracts xsum, rescales and stores.
 // Every CTA stages the whole of x~ (M x K bytes, from L2): at 16 tokens and
 // K = 8640 that is 138 KB per CTA, 20 MB of L2 reads per launch, three
 // times the weight bytes, which is why the kernel stops at 16 tokens (32
@@ -66,11 +69,14 @@ struct MmaDecodeArgs {
 // Slots per token, padded to 4 mod 8 (see above).
 __host__ __device__ constexpr int mma_slot_stride(int nw) { return ((nw + 3) / 8) * 8 + 4; }
 
+// Words per token of the partial tiles: the CTA's 16 RBK rows, plus 4.
+__host__ __device__ constexpr int mma_part_stride(int rbk) { return 16 * rbk + 4; }
+
 // Shared memory: NT8 * 8 tokens x stride slots of 16 bytes, then the partial
-// tiles: RBK blocks x KP parts x 16 rows x NT8 * 8 tokens int32.
+// tiles: KP = 16 / RBK parts x NT8 * 8 tokens x mma_part_stride(RBK) int32.
 __host__ __device__ constexpr size_t mma_decode_smem(int nt8, int rbk, int K) {
   return static_cast<size_t>(nt8) * 8 * mma_slot_stride(K / 16) * 16 +
-         static_cast<size_t>(16) * 16 * nt8 * 8 * 4;
+         static_cast<size_t>(16 / rbk) * nt8 * 8 * mma_part_stride(rbk) * 4;
 }
 
 __device__ __forceinline__ void mma_s8_16832(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
@@ -185,15 +191,16 @@ __global__ void __launch_bounds__(kMmaThreads, 1) k_decode_mma(const MmaDecodeAr
     }
   }
   // C fragment: c0, c1 = row g, tokens 2q, 2q+1; c2, c3 = row g + 8.
-  // part[rb][kp][row 16][token T]
-  int32_t* pp = part + (static_cast<size_t>(rb) * KP + kp) * 16 * T;
+  // part[kp][token T][CTA row, stride PS]
+  constexpr int PS = mma_part_stride(RBK);
+  int32_t* pp = part + static_cast<size_t>(kp) * T * PS + 16 * rb + g;
 #pragma unroll
   for (int n = 0; n < NT8; ++n) {
     const int t0 = 8 * n + 2 * q;
-    pp[g * T + t0] = c[n][0];
-    pp[g * T + t0 + 1] = c[n][1];
-    pp[(g + 8) * T + t0] = c[n][2];
-    pp[(g + 8) * T + t0 + 1] = c[n][3];
+    pp[t0 * PS] = c[n][0];
+    pp[(t0 + 1) * PS] = c[n][1];
+    pp[t0 * PS + 8] = c[n][2];
+    pp[(t0 + 1) * PS + 8] = c[n][3];
   }
   __syncthreads();
   // One (row, token) per thread and round: rows fastest, so the stores of a
@@ -201,10 +208,9 @@ __global__ void __launch_bounds__(kMmaThreads, 1) k_decode_mma(const MmaDecodeAr
   for (int e = tid; e < 16 * RBK * T; e += kMmaThreads) {
     const int t = e / (16 * RBK), row = e - t * (16 * RBK);
     if (row >= nrows || t >= M) continue;
-    const int b = row >> 4, r16 = row & 15;
     int32_t tot = 0;
 #pragma unroll
-    for (int k = 0; k < KP; ++k) tot += part[((static_cast<size_t>(b) * KP + k) * 16 + r16) * T + t];
+    for (int k = 0; k < KP; ++k) tot += part[(static_cast<size_t>(k) * T + t) * PS + row];
     const int32_t yi = tot - s_xsum[t];
     const int64_t o = static_cast<int64_t>(t) * a.N + r_begin + row;
     const float yv = rescale(yi, s_scale[t]);

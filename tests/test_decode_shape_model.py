@@ -160,9 +160,9 @@ def test_warp_mma_kernel_shape_picks():
         st = L.bitlinear_decode_mma_shape(M, K, N, sms, buf)
         return None if st == _lib.BL_ERR_UNSUPPORTED else (st, list(buf))
 
-    assert mma(16, 3200, 8640) == (_lib.BL_OK, [16, 4, 4, 13, 59, 147, 68608])
-    assert mma(16, 8640, 3200) == (_lib.BL_OK, [16, 2, 8, 17, 22, 146, 154624])
-    assert mma(9, 3200, 8640) == (_lib.BL_OK, [16, 4, 4, 13, 59, 147, 68608])
+    assert mma(16, 3200, 8640) == (_lib.BL_OK, [16, 4, 4, 13, 59, 147, 69632])
+    assert mma(16, 8640, 3200) == (_lib.BL_OK, [16, 2, 8, 17, 22, 146, 156672])
+    assert mma(9, 3200, 8640) == (_lib.BL_OK, [16, 4, 4, 13, 59, 147, 69632])
     assert mma(8, 3200, 8640) is None       # 8 tokens: the register kernel
     assert mma(17, 3200, 8640) is None      # more than 16 tokens: the tensor-core kernel
     assert mma(16, 8192, 8192) is None      # 32 steps per warp: beyond the register budget
