@@ -341,17 +341,16 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode(const DecodeArgs a) {
         uint32_t word = 0;
         if (m < a.M && w < NW) {
           const uint2 u = *reinterpret_cast<const uint2*>(xsrc + (static_cast<int64_t>(m) * K + 4 * qd) * 2);
-          const float f0 = __uint_as_float(u.x << 16), f1 = __uint_as_float(u.x & 0xFFFF0000u);
-          const float f2 = __uint_as_float(u.y << 16), f3 = __uint_as_float(u.y & 0xFFFF0000u);
-          uint32_t b0, b1, b2, b3;
+          const float f[4] = {__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u),
+                              __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xFFFF0000u)};
+          uint32_t b[4];
           if (eta_bf16) {
-            b0 = code_bits_bf16_r(f0, eta, heta, qs, rr); b1 = code_bits_bf16_r(f1, eta, heta, qs, rr);
-            b2 = code_bits_bf16_r(f2, eta, heta, qs, rr); b3 = code_bits_bf16_r(f3, eta, heta, qs, rr);
+            code_bits_bf16_n<4>(f, b, eta, heta, qs, rr);
           } else {
-            b0 = quantise_exact_bits(f0, eta); b1 = quantise_exact_bits(f1, eta);
-            b2 = quantise_exact_bits(f2, eta); b3 = quantise_exact_bits(f3, eta);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) b[i] = quantise_exact_bits(f[i], eta);
           }
-          word = pack_lowbytes(b0, b1, b2, b3);
+          word = pack_lowbytes(b[0], b[1], b[2], b[3]);
           psum = __dp4a(static_cast<int>(word), 0x01010101, psum);
           if (a.xq_out && blockIdx.x == 0)
             *reinterpret_cast<uint32_t*>(a.xq_out + static_cast<int64_t>(m) * K + 4 * qd) = word;

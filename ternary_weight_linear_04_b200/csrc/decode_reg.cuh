@@ -163,6 +163,8 @@ __global__ void __launch_bounds__(kRegThreads + 64, 2) k_decode_reg(const RegDec
       const uint4 v = x4[c];
       uint32_t lo, hi;
       if (eta_bf16) {
+        // value by value (the grouped tie vote of codes8_bf16 takes more
+        // registers than this kernel's budget leaves, and measured slower)
         const uint32_t u[4] = {v.x, v.y, v.z, v.w};
         uint32_t q[8];
 #pragma unroll
@@ -370,15 +372,9 @@ __global__ void __launch_bounds__(kRegThreads, 1) k_decode_regm(const RegMultiAr
         const uint4 v = x4[c];
         uint32_t lo, hi;
         if (eta_bf16) {
-          const uint32_t u[4] = {v.x, v.y, v.z, v.w};
-          uint32_t q[8];
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            q[2 * k] = code_bits_bf16_r(__uint_as_float(u[k] << 16), eta, heta, qs, rr);
-            q[2 * k + 1] = code_bits_bf16_r(__uint_as_float(u[k] & 0xFFFF0000u), eta, heta, qs, rr);
-          }
-          lo = pack_lowbytes(q[0], q[1], q[2], q[3]);
-          hi = pack_lowbytes(q[4], q[5], q[6], q[7]);
+          const uint2 q8 = codes8_bf16<4>(v, eta, heta, qs, rr);
+          lo = q8.x;
+          hi = q8.y;
         } else {
           const uint2 lh = quantise_chunk_exact(v, eta);
           lo = lh.x;

@@ -357,4 +357,135 @@ __global__ void __launch_bounds__(NT) k_quant_act(const T* __restrict__ x, int64
   }
 }
 
+// The absmax of eight bf16 values (one 16-byte vector) folded into a pair
+// of running maxima: the bf16x2 max of the magnitudes, exact (a selection;
+// a NaN operand yields the other, as fmaxf does).
+__device__ __forceinline__ __nv_bfloat162 absmax8_bf16(__nv_bfloat162 m, const uint4 v) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    __nv_bfloat162 h;
+    const uint32_t a = w[i] & 0x7FFF7FFFu;  // clear both sign bits
+    memcpy(&h, &a, 4);
+    m = __hmax2(m, h);
+  }
+  return m;
+}
+
+// code_bits_bf16_r for N bf16 values at once (a bf16 eta): the candidate
+// and correction run for all N, and the tie test |e| = eta/2 is one vote
+// over the N, so only a group holding an exact tie (rare) takes the branch
+// that applies the tie rule.  Same bits as code_bits_bf16_r value by value.
+template <int N>
+__device__ __forceinline__ void code_bits_bf16_n(const float (&f)[N], uint32_t (&b)[N], float eta,
+                                                 float heta, float s, float r) {
+  bool tie = false;
+#pragma unroll
+  for (int i = 0; i < N; ++i) {
+    const float t = __fmaf_rn(f[i], s, kRneMagic);
+    const float n0 = __fsub_rn(t, kRneMagic);
+    const float e = __fmaf_rn(-n0, eta, __fmul_rn(f[i], 127.0f));
+    b[i] = __float_as_uint(__fmaf_rn(e, r, t));
+    tie |= fabsf(e) == heta;
+  }
+  if (__builtin_expect(tie, 0)) {
+#pragma unroll
+    for (int i = 0; i < N; ++i) b[i] = code_bits_bf16_r(f[i], eta, heta, s, r);
+  }
+}
+
+// The codes of eight bf16 values (one 16-byte vector), packed in order
+// (byte i of the result = code of value i), for a bf16 eta; the tie vote
+// runs over groups of G values (8, or 4 where registers are scarce).
+template <int G = 8>
+__device__ __forceinline__ uint2 codes8_bf16(const uint4 v, float eta, float heta, float s, float r) {
+  static_assert(G == 4 || G == 8, "groups of 4 or 8 values");
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t b[8];
+#pragma unroll
+  for (int g = 0; g < 8 / G; ++g) {
+    float f[G];
+    uint32_t bg[G];
+#pragma unroll
+    for (int i = 0; i < G / 2; ++i) {
+      f[2 * i] = __uint_as_float(w[g * G / 2 + i] << 16);
+      f[2 * i + 1] = __uint_as_float(w[g * G / 2 + i] & 0xFFFF0000u);
+    }
+    code_bits_bf16_n<G>(f, bg, eta, heta, s, r);
+#pragma unroll
+    for (int i = 0; i < G; ++i) b[g * G + i] = bg[i];
+  }
+  return make_uint2(pack_lowbytes(b[0], b[1], b[2], b[3]), pack_lowbytes(b[4], b[5], b[6], b[7]));
+}
+
+// The same eight codes by the IEEE quotient, for a row whose eta is the
+// 1e-5 floor (not a bf16 value).
+__device__ __forceinline__ uint2 codes8_exact(const uint4 v, float eta) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t b[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    b[2 * i] = quantise_exact_bits(__uint_as_float(w[i] << 16), eta);
+    b[2 * i + 1] = quantise_exact_bits(__uint_as_float(w[i] & 0xFFFF0000u), eta);
+  }
+  return make_uint2(pack_lowbytes(b[0], b[1], b[2], b[3]), pack_lowbytes(b[4], b[5], b[6], b[7]));
+}
+
+// bf16 rows read with 16-byte loads (K a multiple of 8, x 16-byte and xq
+// 8-byte aligned): one NT-thread CTA per token row (grid-stride over rows).
+// Each thread keeps its first CV vectors of the row as packed bf16 pairs
+// between the absmax pass and the quantise pass (the whole row for K up to
+// NT * 8 * CV; longer rows read the rest again), so the per-value work is
+// the bf16x2 max, one unpack and the five fp32 operations of the code, and
+// the row sum is one dp4a per four codes.  Same results as k_quant_act.
+template <int NT, int CV>
+__global__ void __launch_bounds__(NT) k_quant_bf16(const __nv_bfloat16* __restrict__ x, int64_t M,
+                                                    int64_t K, int8_t* __restrict__ xq,
+                                                    float* __restrict__ eta_out,
+                                                    int32_t* __restrict__ xsum_out) {
+  __shared__ float redf[NT / 32];
+  __shared__ int32_t redi[NT / 32];
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  const int64_t nv = K >> 3;  // 16-byte vectors per row
+  for (int64_t m = blockIdx.x; m < M; m += gridDim.x) {
+    const uint4* row = reinterpret_cast<const uint4*>(x + m * K);
+    uint2* qrow = reinterpret_cast<uint2*>(xq + m * K);
+    uint4 cache[CV];
+    __nv_bfloat162 mx = __float2bfloat162_rn(0.0f);
+#pragma unroll
+    for (int c = 0; c < CV; ++c) {
+      const int64_t v = threadIdx.x + static_cast<int64_t>(NT) * c;
+      cache[c] = v < nv ? __ldg(row + v) : make_uint4(0, 0, 0, 0);
+      mx = absmax8_bf16(mx, cache[c]);
+    }
+    for (int64_t v = threadIdx.x + static_cast<int64_t>(NT) * CV; v < nv; v += NT)
+      mx = absmax8_bf16(mx, __ldg(row + v));
+    const float amax = block_max_nt<NT>(fmaxf(__low2float(mx), __high2float(mx)), redf);
+    const float eta = fmaxf(amax, 1e-5f);
+    const float r = rcp_approx(eta);
+    const float s = __fmul_rn(127.0f, r);
+    const float heta = __fmul_rn(0.5f, eta);
+    const bool eta_bf16 = is_bf16_value(eta);
+    int32_t sum = 0;
+    auto emit = [&](int64_t v, const uint4 xv) {
+      const uint2 q = eta_bf16 ? codes8_bf16(xv, eta, heta, s, r) : codes8_exact(xv, eta);
+      qrow[v] = q;
+      sum = __dp4a(static_cast<int>(q.x), 0x01010101, sum);
+      sum = __dp4a(static_cast<int>(q.y), 0x01010101, sum);
+    };
+#pragma unroll
+    for (int c = 0; c < CV; ++c) {
+      const int64_t v = threadIdx.x + static_cast<int64_t>(NT) * c;
+      if (v < nv) emit(v, cache[c]);
+    }
+    for (int64_t v = threadIdx.x + static_cast<int64_t>(NT) * CV; v < nv; v += NT) emit(v, __ldg(row + v));
+    sum = block_sum_nt<NT>(sum, redi);
+    if (threadIdx.x == 0) {
+      eta_out[m] = eta;
+      xsum_out[m] = sum;
+    }
+  }
+}
+
 }  // namespace bl

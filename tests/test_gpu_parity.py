@@ -473,6 +473,53 @@ def test_quantiser_exact_on_every_bf16_tie():
     np.testing.assert_array_equal(xsum.cpu().numpy(), ref_xsum)
 
 
+# (M, K) reaching every launch shape of the vectorised bf16 quantiser: up to
+# 64 rows one vector of 8 values per thread and 128 / 256 / 512 / 1024
+# threads (K up to 1024 / 2048 / 4096 / 8192), then 1024 threads with four
+# vectors each (K up to 32768, longer rows read again); from 65 rows four
+# vectors per thread and 128 / 256 / 512 / 1024 threads (K up to 4096 /
+# 8192 / 16384 / 32768, longer rows read again; 10000 rows of 64 make CTAs
+# loop over rows).  Ragged K (not a multiple of the threads x 8) in most
+# shapes.
+_QUANT_SHAPES = [(3, 1000), (3, 1024), (5, 2040), (64, 4096), (2, 8192), (7, 8200), (1, 34816),
+                 (65, 4096), (65, 4000), (70, 8192), (66, 16384), (65, 17072), (65, 34816),
+                 (65, 51200), (65, 51208), (4000, 1024), (10000, 64)]
+
+
+@pytest.mark.parametrize("M,K", _QUANT_SHAPES)
+def test_quantiser_every_launch_shape(M, K):
+    """Standalone bf16 quantiser on every launch shape: rows drawn from the
+    bf16 values below a bf16 eta (eta itself, then every value whose 127x/eta
+    is exactly a half-integer, up to half the row, then others at random,
+    all at random positions: exact ties in many 8-value vectors, none in
+    others) and heavy-tailed rows, against the oracle."""
+    rng = np.random.default_rng(9000 + M + K)
+    mant = rng.integers(128, 256, size=min(M, 128))  # many rows repeat these
+    rows = []
+    for m in mant:
+        eta = np.float32(m / 128.0)
+        r = _all_bf16_below(eta)
+        h = 254.0 * r[1:].astype(np.float64) / np.float64(eta)  # exact: 16-bit products
+        tie = 1 + np.flatnonzero((h == np.round(h)) & (np.round(h) % 2 == 1))
+        tie = rng.permutation(tie)[:K // 2]
+        rest = np.setdiff1d(np.arange(1, r.size), tie)
+        fill = rng.choice(rest, size=min(K - 1 - tie.size, rest.size), replace=False)
+        pick = np.concatenate([[0], tie, fill])
+        row = np.zeros(K, np.float32)
+        row[rng.permutation(K)[:pick.size]] = r[pick]
+        rows.append(row)
+    if M > 1:  # a row below the 1e-5 floor of eta: the IEEE-quotient branch
+        bits = rng.integers(0x3000, 0x3727, size=K).astype(np.uint32)
+        rows[-1] = (bits << 16).view(np.float32) * np.where(rng.random(K) < 0.5, -1, 1).astype(np.float32)
+    ties = np.stack(rows)[np.arange(M) % len(rows)]
+    for x in (ties, inputs.draw_activations(rng, M, K, "student_t_outliers", "bf16")):
+        ref_xq, ref_eta, ref_xsum = orc.quant_act(x)
+        xq, eta, xsum = gpu_quant(x, "bf16")
+        np.testing.assert_array_equal(eta.cpu().numpy(), ref_eta)
+        np.testing.assert_array_equal(xq.cpu().numpy(), ref_xq)
+        np.testing.assert_array_equal(xsum.cpu().numpy(), ref_xsum)
+
+
 @pytest.mark.parametrize("group", range(4))
 def test_fused_decode_exact_on_every_bf16_tie(group):
     """The same rows through the fused decode kernel's own quantiser, two

@@ -76,6 +76,36 @@ def test_rmsnorm_quant_many_rows_grid_stride():
     check_rows(torch.from_numpy(x).cuda().to(torch.bfloat16))
 
 
+@pytest.mark.parametrize("K", [8, 64, 3200, 8640])
+def test_rmsnorm_quant_mean_square_on_a_rounding_midpoint(K):
+    """Rows whose mean(x^2) is exactly the midpoint of two consecutive fp32
+    values, or 2^-50 (relative) above it: K/8 values 2^k, K/8 values
+    2^(k-12), optionally K/8 values 2^(k-25), the rest zero, shuffled, random
+    signs, so mean(x^2) = 4^k (1 + 2^-24 (+ 2^-50)) / 8.  The kernel's fp64
+    sum cannot decide these: ms must come out as the tie to even, or rounded
+    up."""
+    rng = np.random.default_rng(K)
+    rows = []
+    for k in (-20, -3, 0, 1, 2, 5, 7, 12, 30):  # most of these scales turn a wrong ms into a wrong eta
+        for extra in (False, True):
+            n = K // 8
+            row = np.zeros(K, np.float32)
+            row[:n] = 2.0 ** k
+            row[n:2 * n] = 2.0 ** (k - 12)
+            if extra:
+                row[2 * n:3 * n] = 2.0 ** (k - 25)
+            rows.append(rng.permutation(row) * rng.choice([-1.0, 1.0], K).astype(np.float32))
+    check_rows(torch.from_numpy(np.stack(rows).astype(np.float32)).cuda().to(torch.bfloat16))
+
+
+def test_rmsnorm_quant_rows_reuse_every_buffer():
+    """Far more rows than resident CTAs: every CTA streams several rows
+    through each of its row buffers."""
+    rng = np.random.default_rng(8)
+    x = inputs.draw_activations(rng, 5000, 64, "student_t_outliers", "bf16")
+    check_rows(torch.from_numpy(x).cuda().to(torch.bfloat16))
+
+
 def test_rmsnorm_quant_empty_and_dtype():
     e = torch.empty((0, 64), dtype=torch.bfloat16, device="cuda")
     xq, eta, xsum = bl.rmsnorm_quant_act(e)
