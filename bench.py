@@ -624,12 +624,12 @@ def layer_kernels(M, m):
     if M <= 2 and bl.fused_decode_ok(M, K):
         return "k_decode (fused)"
     if M <= 8 and bl.decode_regm_shape(M, K, N) is not None:
-        return "k_quant_act + k_decode_regm"
+        return "k_quant_bf16 + k_decode_regm"
     if M <= 16 and bl.decode_mma_shape(M, K, N) is not None:
-        return "k_quant_act + k_decode_mma"
+        return "k_quant_bf16 + k_decode_mma"
     if bl.select_path(M, K, N, m["x_all"], m["packed"], m["x_all"]) == "gemv":
-        return "k_quant_act + k_decode"
-    return "k_quant_act + k_gemm_tc"
+        return "k_quant_bf16 + k_decode"
+    return "k_quant_bf16 + k_gemm_tc"
 
 
 def run_sweep(mats, stream, world, peaks, Ms=(2, 4, 8, 12, 16, 32, 64)):
