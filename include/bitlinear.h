@@ -75,8 +75,9 @@ const char* bitlinear_status_str(bl_status status);
 /* Bytes of the packed ternary matrix: N * ceil(K/4).  0 if N or K < 1. */
 size_t bitlinear_packed_bytes(int64_t N, int64_t K);
 
-/* Bytes of scratch bitlinear_pack_weights needs (256 exponent buckets of
- * 64-bit integers, 2048 bytes).  The caller allocates it, 8-byte aligned. */
+/* Bytes of scratch bitlinear_pack_weights needs (2064: 256 exponent buckets
+ * of 64-bit integers, an fp64 sum and a flag).  The caller allocates it,
+ * 8-byte aligned. */
 size_t bitlinear_pack_workspace_bytes(void);
 
 /*
@@ -94,7 +95,10 @@ size_t bitlinear_pack_workspace_bytes(void);
  *                  Codes past K in the last byte of a row are 01.
  *   gamma     out  one fp32 on the device: max(RN32(RN64(S) / (N*K)),
  *                  1e-5) with S the exact sum of |W| (order-independent,
- *                  so every GPU and the CPU oracle agree to the bit).
+ *                  so every GPU and the CPU oracle agree to the bit).  It
+ *                  is taken from an fp64 sum of |W| when an error bound
+ *                  proves that sum gives this value, else from exact
+ *                  integer sums per exponent; the result is the same.
  *   workspace in   bitlinear_pack_workspace_bytes() bytes of device scratch;
  *                  overwritten; must not be shared by calls that may
  *                  overlap on the GPU.
@@ -119,9 +123,9 @@ bl_status bitlinear_pack_weights(const float* W, int64_t N, int64_t K,
  * and on any row split the shards' packed bytes and gamma are bit-identical
  * to those of the whole matrix.
  *
- * Bucket layout: 256 uint64 (bitlinear_pack_workspace_bytes(), 8-byte
- * aligned).  Bucket b (1..254) holds the sum of the integer significands m
- * (< 2^24) of every |W| = m * 2^(b-150), b the biased fp32 exponent
+ * Bucket layout: 256 uint64 (2048 bytes, 8-byte aligned).  Bucket b
+ * (1..254) holds the sum of the integer significands m (< 2^24) of every
+ * |W| = m * 2^(b-150), b the biased fp32 exponent
  * (subnormals in bucket 1).  Buckets 0 and 255 hold no finite values
  * (NaN/Inf weights are outside the contract).  Two's-complement int64
  * addition of the buckets (what an int64 sum all-reduce does) gives the
@@ -158,9 +162,9 @@ bl_status bitlinear_ternarise_pack(const float* W, int64_t N, int64_t K, const f
  * method.
  *
  * Same arguments, results and errors as bitlinear_pack_weights, minus the
- * workspace: the 2048-byte bucket scratch is a file-scope device array of
- * the library (256 x 64-bit), held on every GPU that loads the library until
- * the process exits.  The call allocates nothing (no cudaMalloc, cudaFree
+ * workspace: the 2064-byte pack scratch (256 x 64-bit buckets, an fp64 sum,
+ * a flag) is a file-scope device array of the library, held on every GPU
+ * that loads the library until the process exits.  The call allocates nothing (no cudaMalloc, cudaFree
  * or allocating library routine).
  *   - Limit: N*K <= 2^40 (the exact sum's 64-bit buckets); larger sizes return
  *     BL_ERR_UNSUPPORTED before anything is launched.

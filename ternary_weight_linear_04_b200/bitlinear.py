@@ -37,6 +37,17 @@ def packed_bytes(N, K):
     return int(_lib.lib().bitlinear_packed_bytes(N, K))
 
 
+def _pack_workspace(workspace, dev):
+    """The caller's pack scratch, checked for size, or a new one."""
+    need = int(_lib.lib().bitlinear_pack_workspace_bytes())
+    if workspace is None:
+        return torch.empty(need, dtype=torch.uint8, device=dev)
+    _require_cuda(workspace)
+    if workspace.numel() * workspace.element_size() < need or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous buffer of at least %d bytes" % need)
+    return workspace
+
+
 def pack_weights(W, stream=None, workspace=None, packed=None, gamma=None):
     """fp32 latent weights (N x K, CUDA) -> (packed uint8 N x ceil(K/4), gamma fp32[1])."""
     _require_cuda(W)
@@ -49,8 +60,7 @@ def pack_weights(W, stream=None, workspace=None, packed=None, gamma=None):
         packed = torch.empty((N, (K + 3) // 4), dtype=torch.uint8, device=dev)
     if gamma is None:
         gamma = torch.empty(1, dtype=torch.float32, device=dev)
-    if workspace is None:
-        workspace = torch.empty(int(L.bitlinear_pack_workspace_bytes()), dtype=torch.uint8, device=dev)
+    workspace = _pack_workspace(workspace, dev)
     check(L.bitlinear_pack_weights(_ptr(W), N, K, _ptr(packed), _ptr(gamma), _ptr(workspace),
                                    _stream(stream)), "bitlinear_pack_weights")
     return packed, gamma
@@ -312,8 +322,7 @@ def pack_weights3(W, stream=None, workspace=None):
     dev = W.device
     packed3 = torch.empty((N, packed3_stride(K)), dtype=torch.uint8, device=dev)
     gamma = torch.empty(1, dtype=torch.float32, device=dev)
-    ws = workspace if workspace is not None else torch.empty(
-        int(_lib.lib().bitlinear_pack_workspace_bytes()), dtype=torch.uint8, device=dev)
+    ws = _pack_workspace(workspace, dev)
     check(_lib.lib().bitlinear_pack_weights3(_ptr(W), N, K, _ptr(packed3), _ptr(gamma), _ptr(ws),
                                              _stream(stream)), "bitlinear_pack_weights3")
     return packed3, gamma

@@ -860,6 +860,41 @@ bl_status launch_quant_bf16(const __nv_bfloat16* x, int64_t M, int64_t K, int8_t
   return launch_quant_bf16_nt<1024, 4>(x, M, K, xq, eta, xsum, grid, s);
 }
 
+// Workspace of the single-matrix pack: the 256 exponent buckets (2048
+// bytes), then the fp64 sum of |W| (8 bytes) and the decision flag (4, +4).
+constexpr size_t kPackWorkspaceBytes = bl::kBuckets * 8 + 16;
+
+// gamma of one whole matrix (count = N*K weights) into *gamma: the fp64 sum
+// of |W| and its proof (k_absmean_f64, k_gamma_decide); the exact buckets
+// (k_absmean_buckets, k_gamma_finalize) run only when the proof fails,
+// their CTAs returning at once otherwise.  ws = kPackWorkspaceBytes of
+// scratch; everything is cleared first.
+bl_status pack_gamma(const float* W, int64_t count, unsigned long long* ws, float* gamma, int sms,
+                     cudaStream_t s) {
+  unsigned long long* buckets = ws;
+  double* acc = reinterpret_cast<double*>(ws + bl::kBuckets);
+  int* decided = reinterpret_cast<int*>(ws + bl::kBuckets + 1);
+  bl::k_zero_u64<<<1, 256, 0, s>>>(ws, static_cast<int>(kPackWorkspaceBytes / 8));
+  bl_status st = launch_status();
+  if (st != BL_OK) return st;
+  int64_t ctas = (count / 4 + 255) / 256;
+  if (ctas > static_cast<int64_t>(sms) * 8) ctas = static_cast<int64_t>(sms) * 8;
+  if (ctas < 1) ctas = 1;
+  bl::k_absmean_f64<<<static_cast<int>(ctas), 256, 0, s>>>(W, count, acc);
+  if ((st = launch_status()) != BL_OK) return st;
+  // Tree height: a thread's adds (at most count / threads + 5, whether or
+  // not W allows 16-byte loads), 5 butterfly levels, 7 adds over the warps,
+  // one atomic add per CTA.
+  const int64_t threads = ctas * 256;
+  const int64_t h = (count + threads - 1) / threads + 5 + 5 + 7 + ctas;
+  bl::k_gamma_decide<<<1, 32, 0, s>>>(acc, count, h, gamma, decided);
+  if ((st = launch_status()) != BL_OK) return st;
+  bl::k_absmean_buckets<<<static_cast<int>(ctas), 256, 0, s>>>(W, count, buckets, decided);
+  if ((st = launch_status()) != BL_OK) return st;
+  bl::k_gamma_finalize<<<1, 32, 0, s>>>(buckets, count, gamma, decided);
+  return launch_status();
+}
+
 }  // namespace
 
 extern "C" {
@@ -1026,7 +1061,7 @@ size_t bitlinear_packed_bytes(int64_t N, int64_t K) {
   return static_cast<size_t>(N) * static_cast<size_t>((K + 3) / 4);
 }
 
-size_t bitlinear_pack_workspace_bytes(void) { return bl::kBuckets * sizeof(unsigned long long); }
+size_t bitlinear_pack_workspace_bytes(void) { return kPackWorkspaceBytes; }
 
 bl_status bitlinear_absmean_buckets(const float* W, int64_t N, int64_t K, void* buckets,
                                    void* stream) {
@@ -1045,7 +1080,7 @@ bl_status bitlinear_absmean_buckets(const float* W, int64_t N, int64_t K, void* 
   int64_t ctas = (count / 4 + 255) / 256;
   if (ctas > static_cast<int64_t>(sms) * 8) ctas = static_cast<int64_t>(sms) * 8;
   if (ctas < 1) ctas = 1;
-  bl::k_absmean_buckets<<<static_cast<int>(ctas), 256, 0, s>>>(W, count, b);
+  bl::k_absmean_buckets<<<static_cast<int>(ctas), 256, 0, s>>>(W, count, b, nullptr);
   return launch_status();
 }
 
@@ -1058,7 +1093,7 @@ bl_status bitlinear_gamma_from_buckets(const void* buckets, int64_t count, float
   const bl_status st = device_info(&sms);
   if (st != BL_OK) return st;
   bl::k_gamma_finalize<<<1, 32, 0, as_stream(stream)>>>(
-      static_cast<const unsigned long long*>(buckets), count, gamma);
+      static_cast<const unsigned long long*>(buckets), count, gamma, nullptr);
   return launch_status();
 }
 
@@ -1085,9 +1120,12 @@ bl_status bitlinear_pack_weights(const float* W, int64_t N, int64_t K, uint8_t* 
   if (N < 1 || K < 1) return BL_ERR_INVALID_ARG;
   if (N > (int64_t{1} << 40) / K) return BL_ERR_UNSUPPORTED;
   if (!aligned(W, 4) || !aligned(workspace, 8) || !aligned(gamma, 4)) return BL_ERR_ALIGNMENT;
-  bl_status st = bitlinear_absmean_buckets(W, N, K, workspace, stream);
+  int sms = 148;
+  bl_status st = device_info(&sms);
   if (st != BL_OK) return st;
-  if ((st = bitlinear_gamma_from_buckets(workspace, N * K, gamma, stream)) != BL_OK) return st;
+  if ((st = pack_gamma(W, N * K, static_cast<unsigned long long*>(workspace), gamma, sms,
+                       as_stream(stream))) != BL_OK)
+    return st;
   return bitlinear_ternarise_pack(W, N, K, gamma, packed, stream);
 }
 
@@ -1135,17 +1173,8 @@ bl_status bitlinear_pack_weights3(const float* W, int64_t N, int64_t K, uint8_t*
   bl_status st = device_info(&sms);
   if (st != BL_OK) return st;
   const cudaStream_t s = as_stream(stream);
-  auto* buckets = static_cast<unsigned long long*>(workspace);
-  bl::k_zero_u64<<<1, 256, 0, s>>>(buckets, bl::kBuckets);
-  if ((st = launch_status()) != BL_OK) return st;
-  const int64_t count = N * K;
-  int64_t ctas = (count / 4 + 255) / 256;
-  if (ctas > static_cast<int64_t>(sms) * 8) ctas = static_cast<int64_t>(sms) * 8;
-  if (ctas < 1) ctas = 1;
-  bl::k_absmean_buckets<<<static_cast<int>(ctas), 256, 0, s>>>(W, count, buckets);
-  if ((st = launch_status()) != BL_OK) return st;
-  bl::k_gamma_finalize<<<1, 32, 0, s>>>(buckets, count, gamma);
-  if ((st = launch_status()) != BL_OK) return st;
+  if ((st = pack_gamma(W, N * K, static_cast<unsigned long long*>(workspace), gamma, sms, s)) != BL_OK)
+    return st;
   const int64_t S = bitlinear_packed3_stride(K);
   int64_t pctas = (N * S + 255) / 256;
   if (pctas > static_cast<int64_t>(sms) * 32) pctas = static_cast<int64_t>(sms) * 32;
@@ -1202,15 +1231,15 @@ bl_status bitlinear_forward3(const int8_t* xq, const float* eta, const int32_t* 
 
 // ------------------------------------------------------------ allocation-free packing
 //
-// Scratch for bitlinear_pack_weights_noalloc: the 256 exponent buckets of
-// the exact |W| sum (2048 bytes), in a file-scope device array instead of a
-// caller buffer.  Every GPU that loads the library holds one copy until the
+// Scratch for bitlinear_pack_weights_noalloc: the pack workspace (the 256
+// exponent buckets of the exact |W| sum, the fp64 sum and its decision flag;
+// 2064 bytes), in a file-scope device array instead of a caller buffer.  Every GPU that loads the library holds one copy until the
 // process exits.  In host code the array's name is only a host-side stand-in
 // for the symbol, so its device address is looked up with
 // cudaGetSymbolAddress, once per device, with that device current.
 namespace {
 
-static __device__ __align__(256) unsigned long long g_pack_scratch[bl::kBuckets];
+static __device__ __align__(256) unsigned long long g_pack_scratch[kPackWorkspaceBytes / 8];
 
 unsigned long long* g_pack_scratch_ptr[kMaxDevices] = {nullptr};
 std::mutex g_pack_scratch_mu;
@@ -1239,27 +1268,18 @@ bl_status bitlinear_pack_weights_noalloc(const float* W, int64_t N, int64_t K, u
                                          float* gamma, void* stream) {
   if (!W || !packed || !gamma) return BL_ERR_INVALID_ARG;
   if (N < 1 || K < 1) return BL_ERR_INVALID_ARG;
-  // The fixed 2048-byte scratch holds 64-bit bucket sums of 24-bit
-  // mantissas: exact for up to 2^40 weights.
+  // The fixed scratch holds 64-bit bucket sums of 24-bit mantissas: exact
+  // for up to 2^40 weights.
   if (N > (int64_t{1} << 40) / K) return BL_ERR_UNSUPPORTED;
   if (!aligned(W, 4) || !aligned(gamma, 4)) return BL_ERR_ALIGNMENT;
   int sms = 148;
   bl_status st = device_info(&sms);
   if (st != BL_OK) return st;
-  unsigned long long* buckets = nullptr;
-  if ((st = pack_scratch_address(&buckets)) != BL_OK) return st;
+  unsigned long long* scratch = nullptr;
+  if ((st = pack_scratch_address(&scratch)) != BL_OK) return st;
   const cudaStream_t s = as_stream(stream);
-  // The shared array keeps the previous call's sums: clear it first.
-  bl::k_zero_u64<<<1, 256, 0, s>>>(buckets, bl::kBuckets);
-  if ((st = launch_status()) != BL_OK) return st;
   const int64_t count = N * K;
-  int64_t ctas = (count / 4 + 255) / 256;
-  if (ctas > static_cast<int64_t>(sms) * 8) ctas = static_cast<int64_t>(sms) * 8;
-  if (ctas < 1) ctas = 1;
-  bl::k_absmean_buckets<<<static_cast<int>(ctas), 256, 0, s>>>(W, count, buckets);
-  if ((st = launch_status()) != BL_OK) return st;
-  bl::k_gamma_finalize<<<1, 32, 0, s>>>(buckets, count, gamma);
-  if ((st = launch_status()) != BL_OK) return st;
+  if ((st = pack_gamma(W, count, scratch, gamma, sms, s)) != BL_OK) return st;
   const int64_t bytes = N * ((K + 3) / 4);
   int64_t pctas = (bytes + 255) / 256;
   if (pctas > static_cast<int64_t>(sms) * 32) pctas = static_cast<int64_t>(sms) * 32;

@@ -202,6 +202,85 @@ def test_gamma_exact_on_hard_sums():
         np.testing.assert_array_equal(packed_h, ref_packed)
 
 
+def _midpoint_matrix(N, K, k, extra, rng):
+    """N*K/8 weights 2^k, N*K/8 weights -2^(k-24), optionally N*K/8 weights
+    2^(k-50), the rest 0, shuffled: mean |W| = 2^k (1 + 2^-24) / 8, the
+    midpoint between two fp32 values (or 2^-50 relative above it)."""
+    n = N * K // 8
+    W = np.zeros(N * K, np.float32)
+    W[:n] = 2.0 ** k
+    W[n:2 * n] = -(2.0 ** (k - 24))
+    if extra:
+        W[2 * n:3 * n] = 2.0 ** (k - 50)
+    return rng.permutation(W).reshape(N, K)
+
+
+@pytest.mark.parametrize("N,K", [(8, 64), (333, 80), (8640, 32)])
+def test_pack_gamma_on_rounding_midpoints(N, K):
+    """Matrices whose mean |W| sits exactly on the midpoint of two fp32
+    values, or 2^-50 (relative) above it: the pack's fp64 sum of |W| cannot
+    decide gamma, so its exact exponent buckets must (the tie to even, or
+    rounded up).  gamma, packed bytes and base-3 bytes bit-exact."""
+    rng = np.random.default_rng(N + K)
+    for k in (-7, 0, 3):
+        for extra in (False, True):
+            W = _midpoint_matrix(N, K, k, extra, rng)
+            ref_packed, ref_gamma, _ = orc.pack_weights(W)
+            t = ref.ternarise(W, ref_gamma)
+            want = np.float32(2.0 ** (k - 3))
+            assert ref_gamma == (np.nextafter(want, np.float32(np.inf)) if extra else want)
+            packed_h, gamma_h, _, _ = gpu_pack(W)
+            assert gamma_h.view(np.uint32) == ref_gamma.view(np.uint32)
+            np.testing.assert_array_equal(packed_h, ref_packed)
+            p3, g3 = bl.pack_weights3(torch.from_numpy(W).cuda())
+            assert np.float32(g3.cpu().numpy()[0]).view(np.uint32) == ref_gamma.view(np.uint32)
+            np.testing.assert_array_equal(p3.cpu().numpy(), ref.pack3(t))
+
+
+def _rd32(x):
+    """The largest fp32 <= the fp64 value x."""
+    f = np.float32(x)
+    return np.nextafter(f, np.float32(-np.inf)) if float(f) > x else f
+
+
+def _around(v, n=64):
+    steps = [v]
+    a = b = v
+    for _ in range(n):
+        a = np.nextafter(a, np.float32(-np.inf))
+        b = np.nextafter(b, np.float32(np.inf))
+        steps += [a, b]
+    return np.array(steps, np.float32)
+
+
+def test_pack_weights_at_the_ternary_threshold():
+    """Weights at every fp32 within 64 ulps of gamma (0.5 + 2^-25) -- above
+    it RN32(w / gamma) exceeds 0.5 -- and of gamma / 2, both signs, in a
+    random matrix; re-placed until gamma (which they move) settles.  The
+    kernels compare w with that threshold instead of dividing: packed bytes
+    and gamma bit-exact, 2-bit and base-3."""
+    rng = np.random.default_rng(12)
+    W = rng.normal(0, 0.02, (96, 1000)).astype(np.float32)
+    g = None
+    for _ in range(30):
+        g0, _ = ref.absmean_gamma(W)
+        vals = np.concatenate([_around(_rd32(float(g0) * (0.5 + 2.0 ** -25))), _around(g0 * np.float32(0.5))])
+        W[0, :vals.size] = vals
+        W[1, :vals.size] = -vals
+        g, _ = ref.absmean_gamma(W)
+        if g == g0:
+            break
+    assert g == g0, "gamma did not settle"
+    ref_packed, ref_gamma, _ = orc.pack_weights(W)
+    t = ref.ternarise(W, ref_gamma)
+    assert np.count_nonzero(t[0, :vals.size]) not in (0, vals.size)  # both sides of the threshold
+    packed_h, gamma_h, _, _ = gpu_pack(W)
+    assert gamma_h.view(np.uint32) == ref_gamma.view(np.uint32)
+    np.testing.assert_array_equal(packed_h, ref_packed)
+    p3, _ = bl.pack_weights3(torch.from_numpy(W).cuda())
+    np.testing.assert_array_equal(p3.cpu().numpy(), ref.pack3(t))
+
+
 # ----------------------------------------------------------------- full-size workloads
 
 def sample_positions(M, N, rng, extra_rows=(), extra_cols=()):

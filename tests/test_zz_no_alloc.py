@@ -2,10 +2,12 @@
 
 bitlinear_pack_weights_noalloc serves callers that may not allocate device
 memory themselves (a host framework that owns all device memory, or a path
-that must not call cudaMalloc); it keeps its 2 KB bucket scratch in a device
-array inside the library instead of a caller buffer.  Its packed bytes and
-gamma must equal bitlinear_pack_weights' bit for bit, on consecutive calls
-(the shared scratch must start from zero each time).  This file is collected
+that must not call cudaMalloc); it keeps its 2 KB pack scratch (exponent
+buckets, an fp64 sum and its decision flag) in a device array inside the
+library instead of a caller buffer.  Its packed bytes and gamma must equal
+bitlinear_pack_weights' bit for bit, on consecutive calls (the shared scratch
+must start from zero each time), also when a matrix needs the exact buckets
+between two that do not.  This file is collected
 last so that a run stopping at its first failure has run everything else.
 """
 import ctypes
@@ -45,7 +47,11 @@ def test_noalloc_pack_matches_pack_on_consecutive_calls():
     assert torch.cuda.is_available(), "GPU test"
     L = _lib.lib()
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    mid = np.zeros(8 * 64, np.float32)  # mean |W| on an fp32 rounding midpoint: exact buckets
+    mid[:64] = 1.0
+    mid[64:128] = -(2.0 ** -24)
     cases = [inputs.make_case(31, 1, 4096, 1000, w_dist="laplace")[0],
+             np.random.default_rng(5).permutation(mid).reshape(8, 64),
              inputs.make_case(32, 1, 3200, 777)[0]]
     for W in cases:  # two calls in a row: the second must not see the first's sums
         Wd = torch.from_numpy(W).cuda()
