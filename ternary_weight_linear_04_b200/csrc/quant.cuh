@@ -437,14 +437,14 @@ __device__ __forceinline__ uint2 codes8_exact(const uint4 v, float eta) {
 // between the absmax pass and the quantise pass (the whole row for K up to
 // NT * 8 * CV; longer rows read the rest again), so the per-value work is
 // the bf16x2 max, one unpack and the five fp32 operations of the code, and
-// the row sum is one dp4a per four codes.  Same results as k_quant_act.
+// the row sum is one dp4a per four codes, added into xsum by one atomic per
+// warp (two block barriers fewer per row).  Same results as k_quant_act.
 template <int NT, int CV>
 __global__ void __launch_bounds__(NT) k_quant_bf16(const __nv_bfloat16* __restrict__ x, int64_t M,
                                                     int64_t K, int8_t* __restrict__ xq,
                                                     float* __restrict__ eta_out,
                                                     int32_t* __restrict__ xsum_out) {
   __shared__ float redf[NT / 32];
-  __shared__ int32_t redi[NT / 32];
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int64_t nv = K >> 3;  // 16-byte vectors per row
@@ -461,8 +461,10 @@ __global__ void __launch_bounds__(NT) k_quant_bf16(const __nv_bfloat16* __restri
     }
     for (int64_t v = threadIdx.x + static_cast<int64_t>(NT) * CV; v < nv; v += NT)
       mx = absmax8_bf16(mx, __ldg(row + v));
+    if (threadIdx.x == 0) xsum_out[m] = 0;  // ordered before the warps' adds by the barriers below
     const float amax = block_max_nt<NT>(fmaxf(__low2float(mx), __high2float(mx)), redf);
     const float eta = fmaxf(amax, 1e-5f);
+    if (threadIdx.x == 0) eta_out[m] = eta;
     const float r = rcp_approx(eta);
     const float s = __fmul_rn(127.0f, r);
     const float heta = __fmul_rn(0.5f, eta);
@@ -480,11 +482,11 @@ __global__ void __launch_bounds__(NT) k_quant_bf16(const __nv_bfloat16* __restri
       if (v < nv) emit(v, cache[c]);
     }
     for (int64_t v = threadIdx.x + static_cast<int64_t>(NT) * CV; v < nv; v += NT) emit(v, __ldg(row + v));
-    sum = block_sum_nt<NT>(sum, redi);
-    if (threadIdx.x == 0) {
-      eta_out[m] = eta;
-      xsum_out[m] = sum;
-    }
+    // The row sum without a block reduction: each warp adds its part with
+    // one atomic (integers, so the order of the adds does not matter).
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
+    if ((threadIdx.x & 31) == 0) atomicAdd(xsum_out + m, sum);
   }
 }
 
