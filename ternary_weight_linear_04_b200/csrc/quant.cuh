@@ -376,16 +376,17 @@ __device__ __forceinline__ __nv_bfloat162 absmax8_bf16(__nv_bfloat162 m, const u
 // and correction run for all N, and the tie test |e| = eta/2 is one vote
 // over the N, so only a group holding an exact tie (rare) takes the branch
 // that applies the tie rule.  Same bits as code_bits_bf16_r value by value.
+// (Host and device: the host check of the rule runs this same code.)
 template <int N>
-__device__ __forceinline__ void code_bits_bf16_n(const float (&f)[N], uint32_t (&b)[N], float eta,
-                                                 float heta, float s, float r) {
+__host__ __device__ __forceinline__ void code_bits_bf16_n(const float (&f)[N], uint32_t (&b)[N],
+                                                          float eta, float heta, float s, float r) {
   bool tie = false;
 #pragma unroll
   for (int i = 0; i < N; ++i) {
-    const float t = __fmaf_rn(f[i], s, kRneMagic);
-    const float n0 = __fsub_rn(t, kRneMagic);
-    const float e = __fmaf_rn(-n0, eta, __fmul_rn(f[i], 127.0f));
-    b[i] = __float_as_uint(__fmaf_rn(e, r, t));
+    const float t = f32_fma(f[i], s, kRneMagic);
+    const float n0 = f32_sub(t, kRneMagic);
+    const float e = f32_fma(-n0, eta, f32_mul(f[i], 127.0f));
+    b[i] = f32_bits(f32_fma(e, r, t));
     tie |= fabsf(e) == heta;
   }
   if (__builtin_expect(tie, 0)) {

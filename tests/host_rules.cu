@@ -8,6 +8,10 @@
 //             2^-21 relative; the hardware approximation is within 1 ulp).
 //   div127  : div127_rn(a) against the IEEE quotient a / 127 for every
 //             normal fp32 a >= 2^-119.
+//   vote    : code_bits_bf16_n (the tie test voted over groups of 4 or 8
+//             values) against code_bits_bf16_r value by value, on the same
+//             values as quant, in two groupings (consecutive values, and
+//             values 997 apart), counting the groups that held a tie.
 // Prints counts; the test requires zero mismatches.
 #include <cmath>
 #include <cstdio>
@@ -78,7 +82,56 @@ static int run_div127() {
   return 0;
 }
 
+template <int G>
+static void vote_groups(const float* xs, long long n, long long stride, float eta, float heta, float s,
+                        float r, long long& checked, long long& bad, long long& tie_groups) {
+  for (long long start = 0; start + G <= n; start += G) {
+    float f[G];
+    uint32_t b[G];
+    bool has_tie = false;
+    for (int i = 0; i < G; ++i) {
+      f[i] = xs[((start + i) * stride) % n];
+      volatile float a = f[i] * 127.0f;
+      volatile float q = a / eta;
+      has_tie |= std::fabs(q - std::trunc(q)) == 0.5f;
+    }
+    bl::code_bits_bf16_n<G>(f, b, eta, heta, s, r);
+    for (int i = 0; i < G; ++i) bad += (b[i] != bl::code_bits_bf16_r(f[i], eta, heta, s, r));
+    checked += G;
+    tie_groups += has_tie;
+  }
+}
+
+static int run_vote() {
+  long long checked = 0, bad = 0, tie_groups = 0;
+  const int exps[] = {-12, 0, 20};
+  static float xs[2 * 0x7F80];
+  for (int E : exps) {
+    for (int m = 128; m < 256; ++m) {
+      const float eta = std::ldexp(static_cast<float>(m) / 128.0f, E);
+      const float heta = eta * 0.5f;
+      for (int k = -1; k <= 1; ++k) {
+        const float r = from_bits(to_bits(1.0f / eta) + k);
+        const float s = bl::f32_mul(127.0f, r);
+        long long n = 0;
+        for (uint32_t bb = 0; bb < 0x7F80u; ++bb) {
+          const float v = from_bits(bb << 16);
+          if (!(v <= eta)) continue;
+          xs[n++] = v;
+          xs[n++] = -v;
+        }
+        vote_groups<8>(xs, n, 1, eta, heta, s, r, checked, bad, tie_groups);
+        vote_groups<4>(xs, n, 1, eta, heta, s, r, checked, bad, tie_groups);
+        vote_groups<8>(xs, n, 997, eta, heta, s, r, checked, bad, tie_groups);
+      }
+    }
+  }
+  printf("vote checked=%lld mismatches=%lld tie_groups=%lld\n", checked, bad, tie_groups);
+  return 0;
+}
+
 int main(int argc, char** argv) {
   if (argc > 1 && strcmp(argv[1], "div127") == 0) return run_div127();
+  if (argc > 1 && strcmp(argv[1], "vote") == 0) return run_vote();
   return run_quant();
 }

@@ -5,6 +5,9 @@
   from an approximate reciprocal and an exact fma residual.  Checked for
   every bf16 x with |x| <= eta, for every bf16 significand of eta at five
   exponents, with the reciprocal perturbed by up to 8 ulps either way.
+* The same rule with its tie test voted over 4 or 8 values
+  (code_bits_bf16_n, what the quantiser kernels run) against the rule value
+  by value.
 * The rescale's division by 127 (common.cuh, div127_rn): s = RN32(RN32(eta *
   gamma) / 127) of [Production] pipeline step 5, by a correctly rounded
   reciprocal and one fma correction.  Checked against the IEEE quotient for
@@ -49,6 +52,16 @@ def test_bf16_quantiser_rule_is_exact(driver):
     assert c["checked"] > 100_000_000
     assert c["mismatches"] == 0
     assert c["ties"] > 100  # exact .5 ties occur, so the tie branch is exercised
+
+
+def test_voted_tie_rule_matches_the_rule_value_by_value(driver):
+    """code_bits_bf16_n, the form the quantiser kernels run (the tie test
+    voted over groups of 4 or 8 values), gives the same bits as
+    code_bits_bf16_r for every value, in groups with and without ties."""
+    c = _counts(subprocess.run([driver, "vote"], check=True, capture_output=True, text=True).stdout)
+    assert c["checked"] > 10_000_000
+    assert c["mismatches"] == 0
+    assert c["tie_groups"] > 1000
 
 
 def test_division_by_127_is_correctly_rounded(driver):
