@@ -9,6 +9,7 @@
 
 #include <cmath>
 #include <cstdint>
+#include <cstring>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
@@ -321,6 +322,29 @@ __host__ __device__ __forceinline__ float div127_rn(float a) {
 #else
   const float q0 = a * kInv127;
   return fmaf(fmaf(-q0, 127.0f, a), kInv127, q0);
+#endif
+}
+
+// The fp64 value with high word hi and low word lo (host and device).
+__host__ __device__ __forceinline__ double f64_from_words(uint32_t hi, uint32_t lo) {
+#ifdef __CUDA_ARCH__
+  return __hiloint2double(static_cast<int>(hi), static_cast<int>(lo));
+#else
+  const uint64_t u = (static_cast<uint64_t>(hi) << 32) | lo;
+  double d;
+  memcpy(&d, &u, 8);
+  return d;
+#endif
+}
+
+// RD32(x): the largest fp32 not above the fp64 x (host and device).
+__host__ __device__ __forceinline__ float f32_rd(double x) {
+#ifdef __CUDA_ARCH__
+  return __double2float_rd(x);
+#else
+  float f = static_cast<float>(x);  // nearest
+  if (static_cast<double>(f) > x) f = nextafterf(f, -INFINITY);
+  return f;
 #endif
 }
 

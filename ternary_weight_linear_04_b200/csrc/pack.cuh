@@ -162,9 +162,20 @@ __global__ void k_gamma_finalize(const unsigned long long* __restrict__ buckets,
 //     Otherwise (S within about h 2^-53 of a rounding boundary of gamma)
 //     the buckets run.
 
-__device__ __forceinline__ double widen_f32_mag(uint32_t u) {
+// (The widening helpers and the ternary threshold below are host callable:
+// a host test checks them on every fp32 / bf16 magnitude and against IEEE
+// division.)
+__host__ __device__ __forceinline__ double widen_f32_mag(uint32_t u) {
   const uint32_t a = u & 0x7FFFFFFFu;
-  return __hiloint2double(static_cast<int>((a >> 3) + 0x38000000u), static_cast<int>(a << 29));
+  return f64_from_words((a >> 3) + 0x38000000u, a << 29);
+}
+
+// The fp64 value of a bf16 magnitude (the low 15 bits of h), built the same
+// way: exponent field + 896 (1023 - 127), significand bits moved up.  Exact
+// for normal values; zeros and subnormals (exponent field 0) come out as a
+// wrong value below 2^-126.
+__host__ __device__ __forceinline__ double widen_bf16_mag(uint32_t h) {
+  return f64_from_words(((h & 0x7FFFu) << 13) + 0x38000000u, 0u);
 }
 
 // *acc += sum |W| in fp64 (grid-stride, 16-byte loads when W allows).
@@ -230,11 +241,11 @@ __global__ void k_gamma_decide(const double* __restrict__ acc, int64_t count, in
 // T = gamma * (0.5 + 2^-25) -- exact in fp64: 24 x 25 significant bits --
 // t = +1 iff w > T and -1 iff w < -T.  For an fp32 w, w > T iff w > RD32(T).
 // One comparison per weight replaces the IEEE division.
-__device__ __forceinline__ float ternary_threshold(float gamma) {
-  return __double2float_rd(__dmul_rn(static_cast<double>(gamma), 0.5 + 0x1p-25));
+__host__ __device__ __forceinline__ float ternary_threshold(float gamma) {
+  return f32_rd(static_cast<double>(gamma) * (0.5 + 0x1p-25));  // the product is exact
 }
 
-__device__ __forceinline__ uint32_t ternary_code(float w, float thr) {
+__host__ __device__ __forceinline__ uint32_t ternary_code(float w, float thr) {
   return (w > thr) ? 2u : ((w < -thr) ? 0u : 1u);
 }
 

@@ -28,14 +28,6 @@ namespace bl {
 constexpr int kRowsThreads = 256;
 constexpr int kRowsMaxStages = 4;
 
-// The fp64 value of a bf16 magnitude (the low 15 bits of h), built from its
-// bit pattern: exponent field + 896 (1023 - 127), significand bits moved up.
-// Exact for normal values; zeros and subnormals (exponent field 0) come out
-// as a wrong value below 2^-126.
-__device__ __forceinline__ double widen_bf16_mag(uint32_t h) {
-  return __hiloint2double(static_cast<int>(((h & 0x7FFFu) << 13) + 0x38000000u), 0);
-}
-
 // The 8 fp32 codes of quantise_fast for one vector of bf16 x times the
 // RMSNorm scale r (x_norm = RN32(x * r)), packed in order; the near-tie test
 // is one vote over the 8 values, so only a vector holding a near tie takes
@@ -76,9 +68,10 @@ __device__ __forceinline__ float mean_square_f32(double S, double Kd) {
 // memory.  Same readings and results as k_rmsnorm_quant; the sum of
 // squares S is found in fp64 and proved rather than summed exactly:
 //   * every x^2 of a bf16 x has at most 16 significant bits, so the square
-//     of its fp64 widening (widen_bf16_mag) is exact, and one DFMA adds it
-//     with a single rounding; zeros and subnormals widen to values below
-//     2^-126, whose squares (below 2^-252) stand for 0 or the true square;
+//     of its fp64 widening (widen_bf16_mag, pack.cuh) is exact, and one
+//     DFMA adds it with a single rounding; zeros and subnormals widen to
+//     values below 2^-126, whose squares (below 2^-252) stand for 0 or the
+//     true square;
 //   * S^ = the fp64 sum (per thread, then a warp butterfly, then thread 0
 //     over the warps): a sum of non-negative terms over a tree of height h
 //     is within gamma_h = h u / (1 - h u) (u = 2^-53) of the exact sum of

@@ -1,6 +1,6 @@
-// Host driver for two division-free rules of the kernels, compiled from the
-// kernels' own __host__ __device__ routines (quant.cuh, common.cuh), used by
-// tests/test_fast_rules.py.
+// Host driver for the division-free rules of the kernels, compiled from the
+// kernels' own __host__ __device__ routines (quant.cuh, pack.cuh,
+// common.cuh), used by tests/test_fast_rules.py.
 //   quant   : code_bits_bf16_r against RNE(RN32(RN32(127 x) / eta)) (IEEE
 //             division) for every bf16 x with |x| <= eta, eta = every bf16
 //             significand at several exponents, and reciprocals r that are
@@ -12,11 +12,19 @@
 //             values) against code_bits_bf16_r value by value, on the same
 //             values as quant, in two groupings (consecutive values, and
 //             values 997 apart), counting the groups that held a tie.
+//   widen   : widen_f32_mag on every fp32 magnitude pattern and
+//             widen_bf16_mag on every bf16 one: the exact value for normal
+//             values, a value in [2^-127, 2^-126) for exponent field 0.
+//   thresh  : ternary_code(w, ternary_threshold(gamma)) against
+//             Clip(RNE(RN32(w / gamma)), -1, 1) (IEEE division) for 4096
+//             values of gamma and every fp32 w within 64 ulps of
+//             +-gamma (0.5 + 2^-25), of +-gamma / 2 and of +-1.5 gamma.
 // Prints counts; the test requires zero mismatches.
 #include <cmath>
 #include <cstdio>
 #include <cstring>
 
+#include "pack.cuh"
 #include "quant.cuh"
 
 static float from_bits(uint32_t u) {
@@ -130,8 +138,65 @@ static int run_vote() {
   return 0;
 }
 
+static int run_widen() {
+  long long bad = 0, checked = 0, zero_field = 0;
+#pragma omp parallel for reduction(+ : bad, checked, zero_field) schedule(static)
+  for (long long u = 0; u < 0x80000000LL; ++u) {
+    const uint32_t a = static_cast<uint32_t>(u);
+    const double w = bl::widen_f32_mag(a | 0x80000000u);  // the sign is ignored
+    if ((a >> 23) == 0) {
+      bad += !(w >= 0x1p-127 && w < 0x1p-126);
+      ++zero_field;
+    } else if ((a >> 23) != 0xFF) {
+      bad += (w != static_cast<double>(from_bits(a)));
+    }
+    ++checked;
+  }
+  for (uint32_t h = 0; h < 0x10000u; ++h) {
+    const double w = bl::widen_bf16_mag(h);
+    const uint32_t e = (h >> 7) & 0xFFu;
+    if (e == 0) bad += !(w >= 0x1p-127 && w < 0x1p-126);
+    else if (e != 0xFF) bad += (w != static_cast<double>(std::fabs(from_bits(h << 16))));
+    ++checked;
+  }
+  printf("widen checked=%lld mismatches=%lld zero_field=%lld\n", checked, bad, zero_field);
+  return 0;
+}
+
+static int run_thresh() {
+  long long bad = 0, checked = 0, nonzero = 0;
+  uint32_t state = 12345u;
+  for (int i = 0; i < 4096; ++i) {
+    state = state * 1664525u + 1013904223u;
+    // gamma: 1e-5 .. about 1e5, every significand pattern reachable
+    const float gamma = std::ldexp(1.0f + static_cast<float>(state >> 9) * 0x1p-23f, -17 + static_cast<int>(i % 34));
+    const float thr = bl::ternary_threshold(gamma);
+    const float centers[3] = {static_cast<float>(static_cast<double>(gamma) * (0.5 + 0x1p-25)), gamma * 0.5f,
+                              gamma * 1.5f};
+    for (float c : centers) {
+      for (int k = -64; k <= 64; ++k) {
+        for (int sg = 0; sg < 2; ++sg) {
+          const float w0 = from_bits(to_bits(c) + k);
+          const float w = sg ? -w0 : w0;
+          volatile float q = w / gamma;
+          const float t = std::fmin(1.0f, std::fmax(-1.0f, std::nearbyint(q)));
+          const int want = static_cast<int>(t) + 1;
+          const int got = static_cast<int>(bl::ternary_code(w, thr));
+          bad += (got != want);
+          nonzero += (want != 1);
+          ++checked;
+        }
+      }
+    }
+  }
+  printf("thresh checked=%lld mismatches=%lld nonzero=%lld\n", checked, bad, nonzero);
+  return 0;
+}
+
 int main(int argc, char** argv) {
   if (argc > 1 && strcmp(argv[1], "div127") == 0) return run_div127();
   if (argc > 1 && strcmp(argv[1], "vote") == 0) return run_vote();
+  if (argc > 1 && strcmp(argv[1], "widen") == 0) return run_widen();
+  if (argc > 1 && strcmp(argv[1], "thresh") == 0) return run_thresh();
   return run_quant();
 }
