@@ -12,6 +12,7 @@ import torch
 
 from oracle import native as orc
 from oracle import reference as ref
+from ternary_weight_linear_04_b200 import _lib
 from ternary_weight_linear_04_b200 import bitlinear as bl
 from ternary_weight_linear_04_b200 import build as libbuild
 from ternary_weight_linear_04_b200 import inputs
@@ -235,6 +236,19 @@ def test_pack_gamma_on_rounding_midpoints(N, K):
             p3, g3 = bl.pack_weights3(torch.from_numpy(W).cuda())
             assert np.float32(g3.cpu().numpy()[0]).view(np.uint32) == ref_gamma.view(np.uint32)
             np.testing.assert_array_equal(p3.cpu().numpy(), ref.pack3(t))
+
+
+def test_pack_rejects_a_short_workspace():
+    """The binding checks a caller's pack workspace against
+    bitlinear_pack_workspace_bytes() (the C ABI takes a plain pointer and
+    cannot); a workspace of exactly that size works."""
+    W = torch.zeros((4, 64), device="cuda")
+    with pytest.raises(ValueError):
+        bl.pack_weights(W, workspace=torch.empty(2048, dtype=torch.uint8, device="cuda"))
+    need = int(_lib.lib().bitlinear_pack_workspace_bytes())
+    packed, gamma = bl.pack_weights(W, workspace=torch.empty(need, dtype=torch.uint8, device="cuda"))
+    assert np.float32(gamma.cpu().numpy()[0]) == np.float32(1e-5)  # all-zero W: the floor
+    assert np.all(packed.cpu().numpy() == 0x55)  # every code 01 (t = 0)
 
 
 def _rd32(x):
